@@ -1,0 +1,334 @@
+// rrs_api.cu -- the extern "C" entry points declared in include/rrs.h:
+// argument validation on the host, then stream-ordered kernel launches.
+// No entry point allocates memory; only rrs_check_workspace and
+// rrs_linear_from_host synchronise the host.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include "rrs.h"
+#include "rrs_device.cuh"
+#include "rrs_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "no error";
+
+rrs_status fail(rrs_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+rrs_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(RRS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxK = 32768;
+constexpr int kMaxHadamard = 8192;
+constexpr size_t kWorkspaceBytes = 256;
+
+#define RRS_REQUIRE_PTR(p)                                                          \
+    do {                                                                            \
+        if ((p) == nullptr) return fail(RRS_ERR_INVALID_ARG, "%s is null", #p);     \
+        if (!aligned16(p))                                                          \
+            return fail(RRS_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);      \
+    } while (0)
+
+rrs_status check_K(int K) {
+    if (K < 128 || K % 128 != 0)
+        return fail(K > 0 && K % 2 == 0 ? RRS_ERR_UNSUPPORTED : RRS_ERR_INVALID_ARG,
+                    "K = %d: the CUDA path needs K a positive multiple of 128", K);
+    if (K > kMaxK) return fail(RRS_ERR_UNSUPPORTED, "K = %d exceeds the limit %d", K, kMaxK);
+    return RRS_OK;
+}
+
+// Resolves the Hadamard block size (1 under RRS_NO_ROTATE) and its scale.
+rrs_status check_hadamard(int K, int had_block, unsigned flags, int* n, float* c_n) {
+    int nn = (flags & RRS_NO_ROTATE) ? 1 : had_block;
+    if (nn < 1 || (nn & (nn - 1)) != 0)
+        return fail(RRS_ERR_INVALID_ARG, "had_block = %d is not a power of two", had_block);
+    if (nn > kMaxHadamard)
+        return fail(RRS_ERR_UNSUPPORTED, "had_block = %d exceeds %d", nn, kMaxHadamard);
+    if (K % nn != 0) return fail(RRS_ERR_INVALID_ARG, "K = %d is not a multiple of had_block = %d", K, nn);
+    *n = nn;
+    *c_n = (float)(1.0 / std::sqrt((double)nn));
+    return RRS_OK;
+}
+
+rrs_status check_G(int K, int G) {
+    if (G < 1 || K % G != 0) return fail(RRS_ERR_INVALID_ARG, "G = %d does not divide K = %d", G, K);
+    if (G % 128 != 0) return fail(RRS_ERR_UNSUPPORTED, "G = %d: the CUDA path needs G %% 128 == 0", G);
+    return RRS_OK;
+}
+
+rrs_status check_ws(void* ws, size_t ws_bytes) {
+    if (ws == nullptr || ws_bytes < kWorkspaceBytes)
+        return fail(RRS_ERR_WORKSPACE, "workspace %p of %zu bytes, need %zu", ws, ws_bytes, kWorkspaceBytes);
+    if (!aligned16(ws)) return fail(RRS_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    return RRS_OK;
+}
+
+rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float c_n, const int32_t* perm,
+                               uint8_t* qX, float* s, float* scale_t, unsigned flags, cudaStream_t st) {
+    const int unit = (flags & RRS_FORCE_UNIT_SCALES) ? 1 : 0;
+    rrs::PrepLaunch pl{};
+    pl.X = X;
+    pl.rows = M;
+    pl.K = K;
+    pl.n = n;
+    pl.G = G;
+    pl.c_n = c_n;
+    pl.perm = perm;
+    if (!unit) {
+        cudaError_t e = cudaMemsetAsync(s, 0, sizeof(float) * (size_t)(K / G), st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(s)");
+        pl.mode = 1;
+        pl.max_out = reinterpret_cast<uint32_t*>(s);
+        e = rrs::launch_prep(pl, st);
+        if (e != cudaSuccess) return cuda_fail(e, "group-max kernel");
+    }
+    pl.mode = 0;
+    pl.max_out = nullptr;
+    pl.unit_scales = unit;
+    pl.s_in = s;
+    pl.q_out = qX;
+    pl.scale_out = scale_t;
+    pl.s_unit_out = unit ? s : nullptr;
+    cudaError_t e = rrs::launch_prep(pl, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantise kernel");
+    return RRS_OK;
+}
+
+rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
+                               const float* scale_w, int M, int N, int K, int G, float* Y, int32_t* P,
+                               void* ws, cudaStream_t st) {
+    rrs::GemmLaunch gl{};
+    gl.qX = qX;
+    gl.qW = qW;
+    gl.s = s;
+    gl.scale_t = scale_t;
+    gl.scale_w = scale_w;
+    gl.M = M;
+    gl.N = N;
+    gl.K = K;
+    gl.G = G;
+    gl.Y = Y;
+    gl.P = P;
+    gl.err = reinterpret_cast<uint32_t*>(ws);
+    cudaError_t e = rrs::launch_gemm(gl, st);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM kernel");
+    return RRS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags) {
+    (void)M;
+    (void)N;
+    (void)K;
+    (void)G;
+    (void)had_block;
+    (void)flags;
+    return kWorkspaceBytes;
+}
+
+rrs_status rrs_prepare_weights(const void* W, int N, int K, int had_block, const int32_t* perm, uint8_t* qW,
+                               float* scale_w, unsigned flags, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(W);
+    RRS_REQUIRE_PTR(perm);
+    RRS_REQUIRE_PTR(qW);
+    RRS_REQUIRE_PTR(scale_w);
+    if (N < 1) return fail(RRS_ERR_INVALID_ARG, "N = %d", N);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    rrs::PrepLaunch pl{};
+    pl.X = W;
+    pl.rows = N;
+    pl.K = K;
+    pl.n = n;
+    pl.G = K;
+    pl.c_n = c_n;
+    pl.perm = perm;
+    pl.mode = 0;
+    pl.unit_scales = 1;
+    pl.q_out = qW;
+    pl.scale_out = scale_w;
+    cudaError_t e = rrs::launch_prep(pl, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "weight prep kernel");
+    return RRS_OK;
+}
+
+rrs_status rrs_smooth_quant(const void* X, int M, int K, int G, int had_block, const int32_t* perm, uint8_t* qX,
+                            float* s, float* scale_t, void* ws, size_t ws_bytes, unsigned flags,
+                            rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(X);
+    RRS_REQUIRE_PTR(perm);
+    RRS_REQUIRE_PTR(qX);
+    RRS_REQUIRE_PTR(s);
+    RRS_REQUIRE_PTR(scale_t);
+    if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    r = check_ws(ws, ws_bytes);
+    if (r != RRS_OK) return r;
+    return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, s, scale_t, flags,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
+                         const float* scale_w, int M, int N, int K, int G, float* Y, void* ws, size_t ws_bytes,
+                         rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(qX);
+    RRS_REQUIRE_PTR(s);
+    RRS_REQUIRE_PTR(scale_t);
+    RRS_REQUIRE_PTR(qW);
+    RRS_REQUIRE_PTR(scale_w);
+    RRS_REQUIRE_PTR(Y);
+    if (M < 1 || N < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, N = %d", M, N);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    r = check_ws(ws, ws_bytes);
+    if (r != RRS_OK) return r;
+    return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, const int32_t* perm, int M, int N,
+                      int K, int G, int had_block, uint8_t* qX, float* s, float* scale_t, float* Y, void* ws,
+                      size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
+    if (r != RRS_OK) return r;
+    return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes, stream);
+}
+
+rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* qW, const float* scale_w,
+                                const int32_t* perm, int M, int N, int K, int G, int had_block, uint8_t* qX,
+                                float* s, float* scale_t, float* Y_dev, float* Y_host, void* ws,
+                                size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    if (X_host == nullptr || Y_host == nullptr) return fail(RRS_ERR_INVALID_ARG, "host buffer is null");
+    RRS_REQUIRE_PTR(X_dev);
+    RRS_REQUIRE_PTR(Y_dev);
+    if (M < 1 || N < 1 || K < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, N = %d, K = %d", M, N, K);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(X_dev, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy of X");
+    rrs_status r = rrs_linear(X_dev, qW, scale_w, perm, M, N, K, G, had_block, qX, s, scale_t, Y_dev, ws,
+                              ws_bytes, flags, stream);
+    if (r != RRS_OK) return r;
+    e = cudaMemcpyAsync(Y_host, Y_dev, (size_t)M * N * 4, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy of Y");
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    return RRS_OK;
+}
+
+rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, int M, int N, int K, int G,
+                                        int32_t* P, void* ws, size_t ws_bytes, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(qX);
+    RRS_REQUIRE_PTR(qW);
+    RRS_REQUIRE_PTR(P);
+    if (M < 1 || N < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, N = %d", M, N);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    r = check_ws(ws, ws_bytes);
+    if (r != RRS_OK) return r;
+    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+rrs_status rrs_channel_absmax(const void* X, int M, int K, int had_block, float* cmax, unsigned flags,
+                              rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(X);
+    RRS_REQUIRE_PTR(cmax);
+    if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(cmax, 0, sizeof(float) * (size_t)K, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(cmax)");
+    rrs::PrepLaunch pl{};
+    pl.X = X;
+    pl.rows = M;
+    pl.K = K;
+    pl.n = n;
+    pl.G = K;
+    pl.c_n = c_n;
+    pl.mode = 2;
+    pl.max_out = reinterpret_cast<uint32_t*>(cmax);
+    e = rrs::launch_prep(pl, st);
+    if (e != cudaSuccess) return cuda_fail(e, "channel-max kernel");
+    return RRS_OK;
+}
+
+rrs_status rrs_perm_from_channel_max(const float* cmax_host, int K, int32_t* perm_host) {
+    if (cmax_host == nullptr || perm_host == nullptr) return fail(RRS_ERR_INVALID_ARG, "null host buffer");
+    if (K < 1) return fail(RRS_ERR_INVALID_ARG, "K = %d", K);
+    std::vector<int32_t> idx((size_t)K);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::stable_sort(idx.begin(), idx.end(),
+                     [&](int32_t a, int32_t b) { return cmax_host[a] > cmax_host[b]; });
+    std::memcpy(perm_host, idx.data(), sizeof(int32_t) * (size_t)K);
+    return RRS_OK;
+}
+
+rrs_status rrs_check_workspace(void* ws, rrs_stream_t stream) {
+    if (ws == nullptr) return fail(RRS_ERR_WORKSPACE, "workspace is null");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the workspace error word");
+    if (word != 0) {
+        const uint32_t zero = 0;
+        e = cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace error word");
+        return fail(RRS_ERR_TIMEOUT, "a kernel gave up on a bounded wait (error word 0x%x)", word);
+    }
+    return RRS_OK;
+}
+
+rrs_status rrs_debug_wait_timeout(int limit_us, void* ws, size_t ws_bytes, rrs_stream_t stream) {
+    rrs_status r = check_ws(ws, ws_bytes);
+    if (r != RRS_OK) return r;
+    if (limit_us < 1 || limit_us > 1000000) return fail(RRS_ERR_INVALID_ARG, "limit_us = %d", limit_us);
+    cudaError_t e = rrs::launch_wait_probe((uint64_t)limit_us * 1000ull, reinterpret_cast<uint32_t*>(ws),
+                                           reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "wait probe kernel");
+    return RRS_OK;
+}
+
+const char* rrs_last_error_string(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,351 @@
+"""Benchmark of the RRS W4A4 linear layer (prep + GEMM) on B200.
+
+A step is one RRS linear (online rotation/reorder/group max/quantise, then
+the group-scaled W4A4 GEMM) on each LLaMA-3-8B projection shape the headline
+metric is quoted on: M=2048 tokens, K=4096, N in {4096 (q/o), 1024 (k/v),
+14336 (gate/up)}, G=128, Hadamard 4096.  Inputs are synthetic (seeded,
+outlier-laden); weights are prepared once, off the timed path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  With torchrun (N > 1) every rank runs its own
+replica (the layer does not shard: replicas only); the time is the max over
+ranks and the value the ops of all ranks over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RRS W4A4 linear TOPS (prep+GEMM) at LLaMA-3-8B shapes; % of INT8 TC peak"
+UNIT = "TOPS"
+N_XSETS = 4            # distinct activation buffers per layer, rotated between steps
+# DRAM bytes per GEMM launch from the ncu capture in profiles/ (None until measured
+# for the current kernel).
+GEMM_TRAFFIC_BYTES = None
+
+
+def peaks():
+    """(int8 dense TOPS, HBM GB/s, source).  INT8 = 2 x the measured bf16 figure
+    (nominal ratio 4.5 / 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return 2.0 * float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 2.0 * 1590.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_ours(args):
+    import datetime
+
+    import activation_smoothing_b200 as rrs
+    from activation_smoothing_b200 import workloads as wl
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    names = args.workload.split(",") if args.workload else wl.HEADLINE
+    layers = [wl.LAYERS[n] for n in names]
+    state = []
+    for L in layers:
+        # calibration draw -> reorder index, on the device (product path)
+        Xc = wl.make_activations(L, sample=1, M=min(L.M, 512)).to(dev)
+        perm = rrs.calibrate_perm(Xc, L.had_block)
+        W = wl.make_weights(L).to(dev)
+        qW, sw = rrs.prepare_weights(W, perm, L.had_block)
+        del W
+        xs = [wl.make_activations(L, sample=2 + i + 10 * rank).to(dev) for i in range(N_XSETS)]
+        st = dict(L=L, perm=perm, qW=qW, sw=sw, xs=xs,
+                  qX=torch.empty((L.M, L.K // 2), dtype=torch.uint8, device=dev),
+                  s=torch.empty(L.K // L.G, dtype=torch.float32, device=dev),
+                  st=torch.empty(L.M, dtype=torch.float32, device=dev),
+                  Y=torch.empty((L.M, L.N), dtype=torch.float32, device=dev),
+                  ws=rrs.make_workspace(L.M, L.N, L.K, L.G, L.had_block, device=dev))
+        state.append(st)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def step(i, events=None):
+        for j, st in enumerate(state):
+            L = st["L"]
+            X = st["xs"][i % N_XSETS]
+            if events is not None:
+                events[j][0].record(stream)
+            rrs.smooth_quant(X, st["perm"], L.G, L.had_block, qX=st["qX"], s=st["s"], scale_t=st["st"],
+                             ws=st["ws"])
+            if events is not None:
+                events[j][1].record(stream)
+            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW"], st["sw"], L.G, Y=st["Y"], ws=st["ws"])
+            if events is not None:
+                events[j][2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    for st in state:
+        rrs.check_workspace(st["ws"])
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in state] for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    ms = t0.elapsed_time(t1)
+    for st in state:
+        rrs.check_workspace(st["ws"])
+
+    prep_ms = [sum(evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(K)) / K for j in range(len(state))]
+    gemm_ms = [sum(evs[i][j][1].elapsed_time(evs[i][j][2]) for i in range(K)) / K for j in range(len(state))]
+
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+
+    ops_step = sum(st["L"].ops for st in state)
+    value = ops_step * K * world / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed.
+    e2e = None
+    if not args.no_e2e:
+        hx = [st["xs"][0].cpu().pin_memory() for st in state]
+        hy = [torch.empty((st["L"].M, st["L"].N), dtype=torch.float32).pin_memory() for st in state]
+        Ke = max(3, min(K, 50))
+
+        def e2e_step():
+            for j, st in enumerate(state):
+                L = st["L"]
+                rrs.linear_from_host(hx[j], st["xs"][1], st["qW"], st["sw"], st["perm"], L.G, L.had_block,
+                                     st["qX"], st["s"], st["st"], st["Y"], hy[j], st["ws"])
+        for _ in range(3):
+            e2e_step()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b)
+        if pg:
+            t = torch.tensor([ems], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": ops_step * Ke * world / (ems * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": sum(st["L"].M * st["L"].K * 2 for st in state),
+               "d2h_bytes_per_step": sum(st["L"].M * st["L"].N * 4 for st in state),
+               "steps": Ke}
+
+    int8_peak, hbm_peak, src = peaks()
+    gemm_ops = sum(st["L"].ops for st in state)
+    gemm_tops = gemm_ops / (sum(gemm_ms) * 1e-3) / 1e12
+    prep_bytes = [2 * st["L"].M * st["L"].K + st["L"].M * st["L"].K // 2 + 4 * st["L"].M + 4 * (st["L"].K // st["L"].G)
+                  for st in state]
+    prep_gbs = sum(prep_bytes) / (sum(prep_ms) * 1e-3) / 1e9
+    launches_per_step = 3 * len(state)      # group-max, quantise, GEMM per layer
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 MMA / fp32 prep",
+        "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights)",
+        "config": {"workload": "+".join(names),
+                   "shapes": [dict(M=st["L"].M, K=st["L"].K, N=st["L"].N, G=st["L"].G, had=st["L"].had_block)
+                              for st in state],
+                   "parallelism": f"replicas{world}",
+                   "l2": f"activations rotate over {N_XSETS} sets per layer; per-step footprint exceeds L2"},
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
+                     "kernel": "rrs gemm_kernel (tcgen05 kind::i8)", "peak_source": src + " (2 x bf16 burst)"},
+        "prep": {"ms_per_layer": [round(x, 5) for x in prep_ms], "algorithmic_GBps": round(prep_gbs, 1),
+                 "hbm_frac": round(prep_gbs / hbm_peak, 4)},
+        "gemm": {"ms_per_layer": [round(x, 5) for x in gemm_ms], "TOPS": round(gemm_tops, 1)},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(layers, budget_s=args.cpu_budget)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def _oracle_sample(layers, rows_per_layer, cols_per_layer=None, seed=0):
+    """Times the oracle on a row sample of each layer; returns (ops, seconds)."""
+    import numpy as np
+
+    import oracle
+    from activation_smoothing_b200 import workloads as wl
+
+    ops, secs = 0, 0.0
+    for j, L in enumerate(layers):
+        r = rows_per_layer
+        ncol = L.N if cols_per_layer is None else min(L.N, cols_per_layer)
+        X = wl.make_activations(L, sample=2)[:r].contiguous()
+        W = wl.make_weights(L, N=ncol)
+        perm = np.arange(L.K, dtype=np.int32)
+        _, qW, sw = oracle.prepare_weights(W, L.had_block, perm)     # offline, untimed
+        t = time.perf_counter()
+        _, qX, s, st = oracle.smooth_quant(X, L.G, L.had_block, perm)
+        oracle.linear_rows(qX, s, st, qW, sw, L.G)
+        secs += time.perf_counter() - t
+        ops += 2 * r * ncol * L.K
+    return ops, secs
+
+
+def cpu_baseline(layers, budget_s=20.0):
+    """The oracle as it stands, single-threaded, on a bounded row sample."""
+    ops, secs = _oracle_sample(layers, 1)
+    rows = max(1, min(64, int(budget_s / max(secs, 1e-6))))
+    ops, secs = _oracle_sample(layers, rows)
+    return {"value": ops / secs / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{rows} token rows of each layer (prep of those rows + their GEMM rows, all N); "
+                      f"weights prepared untimed; single-threaded C", "seconds": round(secs, 2)}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    from activation_smoothing_b200 import workloads as wl
+
+    names = args.workload.split(",") if args.workload else wl.HEADLINE
+    layers = [wl.LAYERS[n] for n in names]
+    # size each step so the whole run stays within about args.cpu_budget seconds
+    per_step = args.cpu_budget / max(1, args.steps + args.warmup)
+    ops1, s1 = _oracle_sample(layers, 1, cols_per_layer=256)
+    cols = max(16, min(max(L.N for L in layers), int(256 * per_step / max(s1, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_sample(layers, 1, cols_per_layer=cols)
+    tot_ops, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        o, s = _oracle_sample(layers, 1, cols_per_layer=cols)
+        tot_ops += o
+        tot_s += s
+    v = tot_ops / tot_s / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s * 1e3 / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32/int (CPU oracle)",
+           "data": "synthetic", "config": {"workload": "+".join(names), "parallelism": "host"},
+           "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": f"per step: 1 token row of each layer, prep + GEMM against {cols} "
+                                      f"output columns; weights prepared untimed"},
+           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="", help="comma-separated layer names (default: headline shapes)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,167 @@
+/*
+ * rrs.h -- C ABI of the Rotated Runtime Smooth (RRS) W4A4 linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on "Rotated Runtime Smooth: Training-Free Activation
+ * Smoother for accurate INT4 inference"):
+ *   - activations X [M, K] are rotated online by a normalised Hadamard
+ *     transform, the weights W [N, K] offline by the same transform
+ *     (summary page, "Approach");
+ *   - the channels of both are permuted by one fixed reorder index, which
+ *     leaves Y = X W^T = sum_i X_i W_i^T unchanged (rebuttal page,
+ *     "Description of the reorder process");
+ *   - each group g of G consecutive reordered channels is divided by its
+ *     runtime scale s_g = max |X'| over all tokens and channels of the group,
+ *     computed at inference and never folded into the weights (summary page,
+ *     "Approach"; rebuttal page, "Novelty": group-wise scales aligned with the
+ *     hardware GEMM);
+ *   - the smoothed activations are quantised per token to symmetric INT4
+ *     (scale_t = amax_t / 7), the weights per output channel (scale_w =
+ *     amax_n / 7, round-to-nearest), and
+ *       Y[t][n] = (sum_g s_g * P_g[t][n]) * scale_t[t] * scale_w[n],
+ *       P_g[t][n] = sum_{k in group g} qX[t][k] * qW[n][k]   (exact int32).
+ *
+ * Arithmetic contract (readings where the pages are silent):
+ *   - Hadamard: fp32, radix-2 stages h = 1, 2, 4, ..., pair (j, j+h) ->
+ *     (a + b, a - b); then one multiply by c_n = (float)(1/sqrt(n)).  n is the
+ *     Hadamard block size; K = B * n gives a block-diagonal rotation; n = 1
+ *     (or RRS_NO_ROTATE) means no rotation (plain Runtime Smooth).
+ *   - reorder after rotation: X'[t][j] = X_rot[t][perm[j]].
+ *   - smoothing is an IEEE fp32 division by s_g (s_g == 0 divides by 1).
+ *   - codes q = clamp(rint(x / scale), -8, 7), round half to even; a scale of 0
+ *     gives all-zero codes.
+ *   - packing: byte i of a row = (q[2i] & 0xF) | (q[2i+1] & 0xF) << 4.
+ *   - the integer stages (codes, s, scale_t, scale_w, P_g) are bit-exact
+ *     functions of the inputs; Y is fp32 with the group sum accumulated in
+ *     fp32 in group order.
+ *
+ * Layouts (all row-major, all device pointers unless stated otherwise):
+ *   X        fp16  [M, K]            W      fp16 [N, K]
+ *   perm     int32 [K]  (a permutation of 0..K-1)
+ *   qX       uint8 [M, K/2]          qW     uint8 [N, K/2]
+ *   s        fp32  [K/G]             scale_t fp32 [M]     scale_w fp32 [N]
+ *   Y        fp32  [M, N]            P      int32 [K/G, M, N] (debug only)
+ *
+ * Ownership: the caller owns every buffer, including the workspace.  The
+ * library allocates no device or host memory and never synchronises the host
+ * except in rrs_check_workspace and rrs_linear_from_host (documented there).
+ * Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ * and outputs are valid when the stream reaches that point.  Calls that share
+ * output buffers or a workspace must be ordered on one stream.
+ *
+ * Errors: every entry point returns an rrs_status; rrs_last_error_string()
+ * gives a thread-local description of the last failure.  Argument checks
+ * happen on the host before anything is enqueued.  Kernels bound every wait
+ * (about one second); a kernel that gives up sets an error word in the
+ * workspace and returns, which rrs_check_workspace reports as
+ * RRS_ERR_TIMEOUT.
+ *
+ * Limits of the CUDA path: K % 128 == 0, K <= 32768; G % 128 == 0 and
+ * K % G == 0 (RRS_ERR_UNSUPPORTED otherwise); n a power of two <= 8192 with
+ * K % n == 0; M, N >= 1; pointers to fp16/uint8/fp32 arrays 16-byte aligned.
+ */
+#ifndef RRS_H
+#define RRS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same type, spelled without CUDA headers). */
+typedef struct CUstream_st *rrs_stream_t;
+
+typedef enum {
+    RRS_OK = 0,
+    RRS_ERR_INVALID_ARG = 1, /* a null/misaligned pointer or an inconsistent size */
+    RRS_ERR_UNSUPPORTED = 2, /* valid for the method, outside this path's limits */
+    RRS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+    RRS_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait */
+    RRS_ERR_WORKSPACE = 5    /* workspace null or smaller than rrs_workspace_size */
+} rrs_status;
+
+/* flags */
+#define RRS_NO_ROTATE 1u         /* identity instead of the Hadamard (plain Runtime Smooth) */
+#define RRS_FORCE_UNIT_SCALES 2u /* s := 1 for every group (A4W4 per-channel scheme, no smoothing) */
+
+/* Bytes of workspace the calls below need for this problem (>= 256).  The
+ * workspace must be zero-filled once before first use; it holds the kernels'
+ * error word and any split-K scratch. */
+size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags);
+
+/* Offline weight path (summary page "Approach"; rebuttal page "Description of
+ * the reorder process"): W' = reorder(rotate_n(W)), scale_w[r] = max_k |W'[r][k]| / 7,
+ * qW = pack(clamp(rint(W' / scale_w), -8, 7)).  W fp16 [N, K] -> qW uint8
+ * [N, K/2], scale_w fp32 [N].  Same n and perm as the activations. */
+rrs_status rrs_prepare_weights(const void *W, int N, int K, int had_block, const int32_t *perm,
+                               uint8_t *qW, float *scale_w, unsigned flags, rrs_stream_t stream);
+
+/* Online activation path (summary page "Approach": rotate, reorder, divide
+ * each group by its runtime max; per-token INT4 quantiser scale = amax / 7):
+ * X fp16 [M, K] -> qX uint8 [M, K/2], s fp32 [K/G], scale_t fp32 [M].
+ * s is computed from all M tokens (two passes over X).  Under
+ * RRS_FORCE_UNIT_SCALES, s is written as 1. */
+rrs_status rrs_smooth_quant(const void *X, int M, int K, int G, int had_block, const int32_t *perm,
+                            uint8_t *qX, float *s, float *scale_t, void *ws, size_t ws_bytes,
+                            unsigned flags, rrs_stream_t stream);
+
+/* Group-scaled W4A4 GEMM (rebuttal page "Novelty": the smoothing scale is
+ * applied group-wise to match the hardware GEMM): exact int32 P_g per group
+ * on the tensor cores, Y = (sum_g s_g * P_g) * scale_t * scale_w in fp32. */
+rrs_status rrs_w4a4_gemm(const uint8_t *qX, const float *s, const float *scale_t, const uint8_t *qW,
+                         const float *scale_w, int M, int N, int K, int G, float *Y, void *ws,
+                         size_t ws_bytes, rrs_stream_t stream);
+
+/* rrs_smooth_quant followed by rrs_w4a4_gemm on one stream, no host sync.
+ * qX, s and scale_t are caller-provided intermediate buffers. */
+rrs_status rrs_linear(const void *X, const uint8_t *qW, const float *scale_w, const int32_t *perm,
+                      int M, int N, int K, int G, int had_block, uint8_t *qX, float *s,
+                      float *scale_t, float *Y, void *ws, size_t ws_bytes, unsigned flags,
+                      rrs_stream_t stream);
+
+/* End-to-end variant for callers holding HOST buffers: copies X_host (fp16
+ * [M, K], ideally pinned) to X_dev, runs rrs_linear, copies Y back into
+ * Y_host (fp32 [M, N]) with cudaMemcpyAsync on `stream`, then synchronises
+ * that stream.  All device buffers are caller-provided. */
+rrs_status rrs_linear_from_host(const void *X_host, void *X_dev, const uint8_t *qW,
+                                const float *scale_w, const int32_t *perm, int M, int N, int K,
+                                int G, int had_block, uint8_t *qX, float *s, float *scale_t,
+                                float *Y_dev, float *Y_host, void *ws, size_t ws_bytes,
+                                unsigned flags, rrs_stream_t stream);
+
+/* Debug: the exact per-group partial sums P [K/G, M, N] (int32) of the same
+ * GEMM, written instead of Y.  For small problems only. */
+rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t *qX, const uint8_t *qW, int M, int N, int K,
+                                        int G, int32_t *P, void *ws, size_t ws_bytes,
+                                        rrs_stream_t stream);
+
+/* Calibration statistic for the reorder index: cmax[k] = max_t |X_rot[t][k]|
+ * (rotation only, no reorder).  cmax fp32 [K]. */
+rrs_status rrs_channel_absmax(const void *X, int M, int K, int had_block, float *cmax,
+                              unsigned flags, rrs_stream_t stream);
+
+/* Host helper: perm = channels sorted by descending cmax_host, ties by lower
+ * channel index.  Both arrays are HOST memory of length K. */
+rrs_status rrs_perm_from_channel_max(const float *cmax_host, int K, int32_t *perm_host);
+
+/* Synchronises `stream`, reads and clears the workspace error word.
+ * Returns RRS_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
+ * last check, RRS_OK otherwise. */
+rrs_status rrs_check_workspace(void *ws, rrs_stream_t stream);
+
+/* Fault-injection hook for tests: launches one kernel that waits on a
+ * barrier nothing will release, with a wait limit of `limit_us`
+ * microseconds (1..1000000).  The kernel records the timeout in the
+ * workspace error word and returns; the context stays usable. */
+rrs_status rrs_debug_wait_timeout(int limit_us, void *ws, size_t ws_bytes, rrs_stream_t stream);
+
+/* Thread-local description of the last non-OK status returned on this thread. */
+const char *rrs_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RRS_H */

@@ -1,0 +1,108 @@
+"""The C-ABI library builds, loads and exports every symbol the header declares;
+host-side argument checks and the host sort work without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rrs.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from activation_smoothing_b200 import build
+    build.build()
+    from activation_smoothing_b200 import _binding
+    return _binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rrs_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_core_calls():
+    names = declared_functions()
+    for n in ("rrs_prepare_weights", "rrs_smooth_quant", "rrs_w4a4_gemm", "rrs_linear"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/rrs.h but not exported"
+
+
+def test_library_is_sm100a_build():
+    from activation_smoothing_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH)
+    assert "--use_fast_math" not in build.FLAGS
+
+
+def test_workspace_size(L):
+    assert L.rrs_workspace_size(2048, 4096, 4096, 128, 4096, 0) >= 256
+
+
+def test_perm_from_channel_max_host(L):
+    rng = np.random.default_rng(0)
+    c = rng.standard_normal(1000).astype(np.float32)
+    c[10] = c[20] = c[30] = 5.0          # ties keep the lower index first
+    perm = np.empty(1000, np.int32)
+    rc = L.rrs_perm_from_channel_max(c.ctypes.data_as(ctypes.c_void_p), 1000,
+                                     perm.ctypes.data_as(ctypes.c_void_p))
+    assert rc == 0
+    np.testing.assert_array_equal(perm, np.argsort(-c, kind="stable"))
+    assert list(perm[:3]) == [10, 20, 30]
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_argument_checks_fail_before_any_launch(L):
+    ok = _fake(0x10000)
+    mis = _fake(0x10008)
+    # null pointer
+    assert L.rrs_prepare_weights(None, 16, 256, 256, ok, ok, ok, 0, None) == 1
+    # misaligned pointer
+    assert L.rrs_prepare_weights(mis, 16, 256, 256, ok, ok, ok, 0, None) == 1
+    assert b"aligned" in L.rrs_last_error_string()
+    # K not a multiple of 128 -> unsupported on the CUDA path
+    assert L.rrs_prepare_weights(ok, 16, 200, 8, ok, ok, ok, 0, None) == 2
+    # Hadamard block not a power of two
+    assert L.rrs_prepare_weights(ok, 16, 256, 96, ok, ok, ok, 0, None) == 1
+    # Hadamard block not dividing K
+    assert L.rrs_prepare_weights(ok, 16, 384, 256, ok, ok, ok, 0, None) == 1
+    ws = ok
+    # G not dividing K -> invalid; G not a multiple of 128 -> unsupported
+    assert L.rrs_smooth_quant(ok, 16, 256, 100, 256, ok, ok, ok, ok, ws, 256, 0, None) == 1
+    assert L.rrs_smooth_quant(ok, 16, 256, 64, 256, ok, ok, ok, ok, ws, 256, 0, None) == 2
+    # workspace too small
+    assert L.rrs_smooth_quant(ok, 16, 256, 128, 256, ok, ok, ok, ok, ws, 8, 0, None) == 5
+    # M < 1
+    assert L.rrs_w4a4_gemm(ok, ok, ok, ok, ok, 0, 16, 256, 128, ok, ws, 256, None) == 1
+    assert L.rrs_debug_wait_timeout(0, ws, 256, None) == 1
+    assert len(L.rrs_last_error_string()) > 0
+
+
+def test_binding_shape_checks_without_gpu():
+    import torch
+    import activation_smoothing_b200 as rrs
+    X = torch.zeros(4, 256, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        rrs.smooth_quant(X, torch.arange(256, dtype=torch.int32), 128, 256)   # host tensors rejected
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "activation_smoothing_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "rrs_oracle" not in src, f

@@ -1,0 +1,249 @@
+"""Parity of the CUDA path with the CPU oracle (needs a B200).
+
+Integer stages (codes/bytes of qX and qW, s, scale_t, scale_w, per-group
+int32 partials) must match bit for bit; Y must satisfy, per element,
+|dY| <= 1e-3 |Y_oracle| + 2^-20 sum_g |s_g P_g| scale_t scale_w.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_smoothing_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda")
+
+
+@pytest.fixture(scope="module")
+def rrs():
+    import activation_smoothing_b200 as m
+    m.lib()
+    return m
+
+
+def bits(t):
+    a = t.detach().cpu().numpy() if isinstance(t, torch.Tensor) else np.asarray(t)
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def assert_bits_equal(gpu, orc, what):
+    g = bits(gpu)
+    o = bits(orc)
+    assert g.shape == o.shape, what
+    bad = np.nonzero(g != o)
+    assert bad[0].size == 0, f"{what}: {bad[0].size} mismatches, first at {[b[0] for b in bad]}"
+
+
+def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
+    """Runs the CUDA path and the oracle on the same inputs and compares."""
+    K = X.shape[1]
+    unit = bool(flags & rrs.FORCE_UNIT_SCALES)
+    n_eff = 1 if flags & rrs.NO_ROTATE else n
+    Xd, Wd, pd = X.to(DEV), W.to(DEV), perm.to(DEV)
+    qW, sw = rrs.prepare_weights(Wd, pd, n, flags)
+    qX, s, st = rrs.smooth_quant(Xd, pd, G, n, flags)
+    ws = rrs.make_workspace(X.shape[0], W.shape[0], K, G, n, flags)
+    Y = rrs.w4a4_gemm(qX, s, st, qW, sw, G, ws=ws)
+    rrs.check_workspace(ws)
+    torch.cuda.synchronize()
+
+    _, oqX, os_, ost = oracle.smooth_quant(X, G, n_eff, perm.numpy(), unit_scales=unit)
+    assert_bits_equal(s, os_, "s")
+    assert_bits_equal(st, ost, "scale_t")
+    assert_bits_equal(qX, oqX, "qX")
+    _, oqW, osw = oracle.prepare_weights(W, n_eff, perm.numpy())
+    assert_bits_equal(sw, osw, "scale_w")
+    assert_bits_equal(qW, oqW, "qW")
+    if check_y:
+        Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
+        Yg = Y.cpu().numpy() if rows is None else Y.cpu().numpy()[rows]
+        ok = oracle.y_tolerance_ok(Yg, Yo, B)
+        assert ok.all(), f"Y: {np.count_nonzero(~ok)} of {ok.size} outside tolerance"
+        rel = np.linalg.norm(Yg - Yo) / max(np.linalg.norm(Yo), 1e-30)
+        assert rel < 1e-5
+    return dict(qX=qX, s=s, st=st, qW=qW, sw=sw, Y=Y)
+
+
+# ------------------------------------------------------------------ tiny ---
+
+@pytest.mark.parametrize("perm_kind", ["identity", "calibrated", "random"])
+def test_tiny_full_parity(rrs, perm_kind):
+    L = wl.LAYERS["tiny"]
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    if perm_kind == "identity":
+        perm = wl.identity_perm(L.K)
+    elif perm_kind == "random":
+        perm = wl.random_perm(L.K, 5)
+    else:
+        perm = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(L, sample=1), L.had_block))
+    run_layer(rrs, X, W, perm, L.G, L.had_block)
+
+
+def test_tiny_partials_bit_exact(rrs):
+    L = wl.LAYERS["tiny"]
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = wl.random_perm(L.K, 9)
+    _, oqX, _, _ = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
+    _, oqW, _ = oracle.prepare_weights(W, L.had_block, perm.numpy())
+    P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(oqX).to(DEV), torch.from_numpy(oqW).to(DEV), L.G)
+    assert_bits_equal(P, oracle.group_partials(oqX, oqW, L.G), "P_g")
+
+
+def test_partials_extreme_codes(rrs):
+    """All codes -8 or 7 (|P_g| at its maximum 64 G) stay exact."""
+    rng = np.random.default_rng(1)
+    M, N, K, G = 130, 136, 512, 256
+    qX = rng.choice(np.array([0x88, 0x77, 0x87, 0x78], np.uint8), size=(M, K // 2))
+    qW = rng.choice(np.array([0x88, 0x77], np.uint8), size=(N, K // 2))
+    qX[3, :] = 0x88
+    qW[5, :] = 0x88
+    P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(qX).to(DEV), torch.from_numpy(qW).to(DEV), G)
+    Po = oracle.group_partials(qX, qW, G)
+    assert Po[0, 3, 5] == 64 * G
+    assert_bits_equal(P, Po, "P_g extreme")
+
+
+def test_tiny_plain_runtime_smooth_and_unit_scales(rrs):
+    L = wl.LAYERS["tiny"]
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = wl.random_perm(L.K, 2)
+    run_layer(rrs, X, W, perm, L.G, L.had_block, flags=rrs.NO_ROTATE)
+    run_layer(rrs, X, W, perm, L.G, 1)
+    r = run_layer(rrs, X, W, perm, L.G, L.had_block, flags=rrs.FORCE_UNIT_SCALES)
+    assert torch.all(r["s"] == 1)
+
+
+# ------------------------------------------------------------ edge cases ---
+
+@pytest.mark.parametrize("M,N,K,G,n", [
+    (1, 256, 256, 128, 256),
+    (17, 136, 512, 128, 64),
+    (130, 200, 1024, 256, 1024),
+    (257, 384, 2048, 2048, 2048),       # one group (G = K)
+    (64, 128, 384, 128, 128),           # K not a power of two, 3 Hadamard blocks
+    (33, 520, 4096, 512, 1),            # no rotation, ragged N
+])
+def test_edge_shapes(rrs, M, N, K, G, n):
+    L = wl.Layer("edge", M, K, N, G, n, seed=M * 7 + N)
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    run_layer(rrs, X, W, wl.random_perm(K, M + N), G, n)
+
+
+def test_zero_group_and_zero_token(rrs):
+    L = wl.Layer("zeros", 40, 512, 256, 128, 512, seed=3)
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    X[7, :] = 0                      # a token that is zero everywhere
+    perm = wl.identity_perm(L.K)
+    # rotated group 2 is zero for all tokens only if the input is zero in a
+    # whole Hadamard block; with no rotation zero channels 256..383 instead
+    X[:, 256:384] = 0
+    r = run_layer(rrs, X, W, perm, L.G, 1)
+    assert r["s"][2].item() == 0 and r["st"][7].item() == 0
+    run_layer(rrs, X, W, perm, L.G, L.had_block)
+
+
+def test_channel_absmax_and_calibrated_perm(rrs):
+    for name in ("tiny", "llama3_8b_qo", "llama3_8b_down"):
+        L = wl.LAYERS[name]
+        Xc = wl.make_activations(L, sample=1, M=min(L.M, 512))
+        cm = rrs.channel_absmax(Xc.to(DEV), L.had_block)
+        assert_bits_equal(cm, oracle.channel_absmax(Xc, L.had_block), f"cmax {name}")
+        perm = rrs.calibrate_perm(Xc.to(DEV), L.had_block)
+        np.testing.assert_array_equal(perm.cpu().numpy(), oracle.calibrate_perm(Xc, L.had_block))
+
+
+# ------------------------------------------------------- full-size layers ---
+
+def _sample_rows(M, st, k=48, seed=0):
+    rng = np.random.default_rng(seed)
+    top = list(np.argsort(-st)[:8])
+    rest = list(rng.choice(M, size=min(M, k), replace=False))
+    return sorted(set(top + rest + [0, M - 1]))
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_kv", "llama3_8b_qo", "llama3_8b_gateup", "llama3_8b_down"])
+def test_llama3_8b_layers(rrs, name):
+    L = wl.LAYERS[name]
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(L, sample=1, M=512), L.had_block))
+    _, _, _, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
+    rows = _sample_rows(L.M, ost, k=24 if L.N > 8192 else 48)
+    run_layer(rrs, X, W, perm, L.G, L.had_block, rows=rows)
+
+
+@pytest.mark.parametrize("name,N", [("llama3_70b_qo_decode_m1", 8192), ("llama3_70b_gateup_decode_m8", 4096),
+                                    ("llama3_70b_down_decode_m16", 2048)])
+def test_llama3_70b_decode(rrs, name, N):
+    """Decode token counts at the 70B K and Hadamard sizes (N cut to keep the
+    oracle's weight path short; N is a plain GEMM dimension)."""
+    L = wl.LAYERS[name]
+    X, W = wl.make_activations(L), wl.make_weights(L, N=N)
+    perm = wl.random_perm(L.K, 1)
+    run_layer(rrs, X, W, perm, L.G, L.had_block, rows=None)
+
+
+def test_llama3_70b_prefill_prep(rrs):
+    """70B q/o prep at full size (M=4096, K=8192, n=8192): codes and scales."""
+    L = wl.LAYERS["llama3_70b_qo"]
+    X = wl.make_activations(L)
+    perm = wl.random_perm(L.K, 4)
+    qX, s, st = rrs.smooth_quant(X.to(DEV), perm.to(DEV), L.G, L.had_block)
+    _, oqX, os_, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
+    assert_bits_equal(s, os_, "s")
+    assert_bits_equal(st, ost, "scale_t")
+    assert_bits_equal(qX, oqX, "qX")
+
+
+@pytest.mark.parametrize("G,n", [(256, 4096), (512, 1), (4096, 4096)])
+def test_group_sweep_shapes(rrs, G, n):
+    L = wl.Layer("sweep", 2048, 4096, 1024, G, n, seed=G + n)
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(L, sample=1, M=256), n))
+    _, _, _, ost = oracle.smooth_quant(X, G, n, perm.numpy())
+    run_layer(rrs, X, W, perm, G, n, rows=_sample_rows(L.M, ost, 16))
+
+
+# ----------------------------------------------------------- API surface ---
+
+def test_linear_equals_two_calls_and_host_path(rrs):
+    L = wl.LAYERS["llama3_8b_kv"]
+    X, W = wl.make_activations(L, M=256), wl.make_weights(L)
+    perm = wl.random_perm(L.K, 8).to(DEV)
+    Xd = X.to(DEV)
+    qW, sw = rrs.prepare_weights(W.to(DEV), perm, L.had_block)
+    qX, s, st = rrs.smooth_quant(Xd, perm, L.G, L.had_block)
+    Y1 = rrs.w4a4_gemm(qX, s, st, qW, sw, L.G)
+    Y2 = rrs.linear(Xd, qW, sw, perm, L.G, L.had_block)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    M, N, K = 256, L.N, L.K
+    Xh = X.pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.float32).pin_memory()
+    ws = rrs.make_workspace(M, N, K, L.G, L.had_block)
+    rrs.linear_from_host(Xh, torch.empty_like(Xd), qW, sw, perm, L.G, L.had_block,
+                         torch.empty_like(qX), torch.empty_like(s), torch.empty_like(st),
+                         torch.empty((M, N), dtype=torch.float32, device=DEV), Yh, ws)
+    assert torch.equal(Yh, Y1.cpu())
+
+
+def test_invalid_arguments_raise(rrs):
+    X = torch.zeros(4, 200, dtype=torch.float16, device=DEV)
+    with pytest.raises(rrs.RRSError) as e:
+        rrs.smooth_quant(X, torch.arange(200, dtype=torch.int32, device=DEV), 100, 8)
+    assert e.value.status_name in ("RRS_ERR_UNSUPPORTED", "RRS_ERR_INVALID_ARG")
+    X = torch.zeros(4, 256, dtype=torch.float16, device=DEV)
+    with pytest.raises(rrs.RRSError) as e:
+        rrs.smooth_quant(X, torch.arange(256, dtype=torch.int32, device=DEV), 64, 256)
+    assert e.value.status_name == "RRS_ERR_UNSUPPORTED"
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(rrs):
+    ws = rrs.make_workspace(16, 16, 256, 128, 256)
+    rrs.debug_wait_timeout(2000, ws)            # 2 ms limit, nothing releases the wait
+    with pytest.raises(rrs.RRSError) as e:
+        rrs.check_workspace(ws)
+    assert e.value.status_name == "RRS_ERR_TIMEOUT"
+    rrs.check_workspace(ws)                     # cleared
+    test_tiny_full_parity(rrs, "identity")      # the context still works
