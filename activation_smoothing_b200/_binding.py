@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "librrs.so")
 
 NO_ROTATE = 1
 FORCE_UNIT_SCALES = 2
+WS_HOLDS_A8 = 4
 
 _STATUS = {
     0: "RRS_OK",
@@ -53,7 +54,7 @@ def lib() -> ctypes.CDLL:
         "rrs_workspace_size": ([I, I, I, I, I, U], Z),
         "rrs_prepare_weights": ([P, I, I, I, P, P, P, U, P], I),
         "rrs_smooth_quant": ([P, I, I, I, I, P, P, P, P, P, Z, U, P], I),
-        "rrs_w4a4_gemm": ([P, P, P, P, P, I, I, I, I, P, P, Z, P], I),
+        "rrs_w4a4_gemm": ([P, P, P, P, P, I, I, I, I, P, P, Z, U, P], I),
         "rrs_linear": ([P, P, P, P, I, I, I, I, I, P, P, P, P, P, Z, U, P], I),
         "rrs_linear_from_host": ([P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, Z, U, P], I),
         "rrs_w4a4_gemm_debug_partials": ([P, P, I, I, I, I, P, P, Z, P], I),
@@ -61,6 +62,7 @@ def lib() -> ctypes.CDLL:
         "rrs_perm_from_channel_max": ([P, I, P], I),
         "rrs_check_workspace": ([P, P], I),
         "rrs_debug_wait_timeout": ([I, P, Z, P], I),
+        "rrs_debug_divide": ([P, P, I, P, P, P], I),
         "rrs_last_error_string": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sigs.items():
@@ -147,8 +149,9 @@ def smooth_quant(X: torch.Tensor, perm: torch.Tensor, G: int, had_block: int, fl
 
 def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torch.Tensor,
               scale_w: torch.Tensor, G: int, Y: Optional[torch.Tensor] = None,
-              ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Group-scaled W4A4 GEMM -> Y fp32 [M, N]."""
+              ws: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
+    """Group-scaled W4A4 GEMM -> Y fp32 [M, N].  flags=WS_HOLDS_A8 when ``ws`` is the
+    workspace the preceding smooth_quant of this qX wrote (skips re-expanding qX)."""
     M, K2 = qX.shape
     N = qW.shape[0]
     K = 2 * K2
@@ -161,7 +164,7 @@ def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torc
     _need(Y, "Y", torch.float32, (M, N))
     ws = make_workspace(M, N, K, G, 1, 0, qX.device) if ws is None else ws
     _check(lib().rrs_w4a4_gemm(_ptr(qX), _ptr(s), _ptr(scale_t), _ptr(qW), _ptr(scale_w), M, N, K, G, _ptr(Y),
-                               _ptr(ws), ws.numel(), _stream(stream)))
+                               _ptr(ws), ws.numel(), flags, _stream(stream)))
     return Y
 
 
@@ -260,3 +263,14 @@ def check_workspace(ws: torch.Tensor, stream=None) -> None:
 def debug_wait_timeout(limit_us: int, ws: torch.Tensor, stream=None) -> None:
     """Launch the fault-injection kernel (a wait that nothing releases, bounded by limit_us)."""
     _check(lib().rrs_debug_wait_timeout(limit_us, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def debug_divide(a: torch.Tensor, b: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(division as the activation kernels compute it, IEEE division) for fp32 device vectors."""
+    n = a.numel()
+    _need(a, "a", torch.float32, (n,))
+    _need(b, "b", torch.float32, (n,))
+    qf = torch.empty_like(a)
+    qi = torch.empty_like(a)
+    _check(lib().rrs_debug_divide(_ptr(a), _ptr(b), n, _ptr(qf), _ptr(qi), _stream(stream)))
+    return qf, qi

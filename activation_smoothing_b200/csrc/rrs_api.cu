@@ -36,7 +36,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int kMaxK = 32768;
 constexpr int kMaxHadamard = 8192;
-constexpr size_t kWorkspaceBytes = 256;
+constexpr size_t kHeaderBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout: [header 256 B: error word] [int8 activation operand, M*K]
+// [fp32 reordered activations X', M*K*4, fast path only].
+size_t ws_a8_offset() { return kHeaderBytes; }
+size_t ws_scratch_offset(int M, int K) { return kHeaderBytes + align256((size_t)M * K); }
+size_t ws_bytes_gemm(int M, int K) { return kHeaderBytes + align256((size_t)M * K); }
+size_t ws_bytes_full(int M, int K, int n) {
+    size_t b = ws_bytes_gemm(M, K);
+    if (rrs::prep_fast_supported(K, n)) b += align256(rrs::prep_fast_scratch_bytes(M, K));
+    return b;
+}
 
 #define RRS_REQUIRE_PTR(p)                                                          \
     do {                                                                            \
@@ -72,16 +85,37 @@ rrs_status check_G(int K, int G) {
     return RRS_OK;
 }
 
-rrs_status check_ws(void* ws, size_t ws_bytes) {
-    if (ws == nullptr || ws_bytes < kWorkspaceBytes)
-        return fail(RRS_ERR_WORKSPACE, "workspace %p of %zu bytes, need %zu", ws, ws_bytes, kWorkspaceBytes);
+rrs_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr || ws_bytes < need)
+        return fail(RRS_ERR_WORKSPACE, "workspace %p of %zu bytes, need %zu (rrs_workspace_size)", ws, ws_bytes, need);
     if (!aligned16(ws)) return fail(RRS_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
     return RRS_OK;
 }
 
 rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float c_n, const int32_t* perm,
-                               uint8_t* qX, float* s, float* scale_t, unsigned flags, cudaStream_t st) {
+                               uint8_t* qX, float* s, float* scale_t, void* ws, unsigned flags, cudaStream_t st) {
     const int unit = (flags & RRS_FORCE_UNIT_SCALES) ? 1 : 0;
+    int8_t* qX8 = reinterpret_cast<int8_t*>(static_cast<unsigned char*>(ws) + ws_a8_offset());
+    if (rrs::prep_fast_supported(K, n)) {
+        rrs::PrepFastLaunch pf{};
+        pf.X = X;
+        pf.rows = M;
+        pf.K = K;
+        pf.n = n;
+        pf.G = G;
+        pf.c_n = c_n;
+        pf.perm = perm;
+        pf.unit_scales = unit;
+        pf.s = s;
+        pf.qX = qX;
+        pf.qX8 = qX8;
+        pf.scale_t = scale_t;
+        pf.scratch = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + ws_scratch_offset(M, K));
+        cudaError_t e = rrs::launch_prep_fast(pf, st);
+        if (e != cudaSuccess) return cuda_fail(e, "rotation/quantise kernels");
+        return RRS_OK;
+    }
+    // General shapes: two passes that each rotate, then the int8 operand.
     rrs::PrepLaunch pl{};
     pl.X = X;
     pl.rows = M;
@@ -107,14 +141,21 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
     pl.s_unit_out = unit ? s : nullptr;
     cudaError_t e = rrs::launch_prep(pl, st);
     if (e != cudaSuccess) return cuda_fail(e, "quantise kernel");
+    e = rrs::launch_expand(qX, qX8, M, K, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expand kernel");
     return RRS_OK;
 }
 
 rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
                                const float* scale_w, int M, int N, int K, int G, float* Y, int32_t* P,
-                               void* ws, cudaStream_t st) {
+                               void* ws, unsigned flags, cudaStream_t st) {
+    int8_t* qX8 = reinterpret_cast<int8_t*>(static_cast<unsigned char*>(ws) + ws_a8_offset());
+    if (!(flags & RRS_WS_HOLDS_A8)) {
+        cudaError_t e = rrs::launch_expand(qX, qX8, M, K, st);
+        if (e != cudaSuccess) return cuda_fail(e, "expand kernel");
+    }
     rrs::GemmLaunch gl{};
-    gl.qX = qX;
+    gl.qX8 = qX8;
     gl.qW = qW;
     gl.s = s;
     gl.scale_t = scale_t;
@@ -136,13 +177,11 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
 extern "C" {
 
 size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags) {
-    (void)M;
     (void)N;
-    (void)K;
     (void)G;
-    (void)had_block;
-    (void)flags;
-    return kWorkspaceBytes;
+    if (M < 1 || K < 1) return kHeaderBytes;
+    const int n = (flags & RRS_NO_ROTATE) ? 1 : had_block;
+    return ws_bytes_full(M, K, n);
 }
 
 rrs_status rrs_prepare_weights(const void* W, int N, int K, int had_block, const int32_t* perm, uint8_t* qW,
@@ -192,15 +231,15 @@ rrs_status rrs_smooth_quant(const void* X, int M, int K, int G, int had_block, c
     float c_n;
     r = check_hadamard(K, had_block, flags, &n, &c_n);
     if (r != RRS_OK) return r;
-    r = check_ws(ws, ws_bytes);
+    r = check_ws(ws, ws_bytes, ws_bytes_full(M, K, n));
     if (r != RRS_OK) return r;
-    return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, s, scale_t, flags,
+    return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, s, scale_t, ws, flags,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
                          const float* scale_w, int M, int N, int K, int G, float* Y, void* ws, size_t ws_bytes,
-                         rrs_stream_t stream) {
+                         unsigned flags, rrs_stream_t stream) {
     RRS_REQUIRE_PTR(qX);
     RRS_REQUIRE_PTR(s);
     RRS_REQUIRE_PTR(scale_t);
@@ -212,9 +251,9 @@ rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t
     if (r != RRS_OK) return r;
     r = check_G(K, G);
     if (r != RRS_OK) return r;
-    r = check_ws(ws, ws_bytes);
+    r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
-    return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws,
+    return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws, flags,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -223,7 +262,7 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
                       size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
-    return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes, stream);
+    return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes, RRS_WS_HOLDS_A8, stream);
 }
 
 rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* qW, const float* scale_w,
@@ -257,9 +296,9 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, in
     if (r != RRS_OK) return r;
     r = check_G(K, G);
     if (r != RRS_OK) return r;
-    r = check_ws(ws, ws_bytes);
+    r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
-    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws,
+    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws, 0u,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -320,12 +359,20 @@ rrs_status rrs_check_workspace(void* ws, rrs_stream_t stream) {
 }
 
 rrs_status rrs_debug_wait_timeout(int limit_us, void* ws, size_t ws_bytes, rrs_stream_t stream) {
-    rrs_status r = check_ws(ws, ws_bytes);
+    rrs_status r = check_ws(ws, ws_bytes, kHeaderBytes);
     if (r != RRS_OK) return r;
     if (limit_us < 1 || limit_us > 1000000) return fail(RRS_ERR_INVALID_ARG, "limit_us = %d", limit_us);
     cudaError_t e = rrs::launch_wait_probe((uint64_t)limit_us * 1000ull, reinterpret_cast<uint32_t*>(ws),
                                            reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "wait probe kernel");
+    return RRS_OK;
+}
+
+rrs_status rrs_debug_divide(const float* a, const float* b, int n, float* q_fast, float* q_ieee,
+                            rrs_stream_t stream) {
+    if (!a || !b || !q_fast || !q_ieee || n < 1) return fail(RRS_ERR_INVALID_ARG, "rrs_debug_divide arguments");
+    cudaError_t e = rrs::launch_divide_check(a, b, n, q_fast, q_ieee, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "divide check kernel");
     return RRS_OK;
 }
 

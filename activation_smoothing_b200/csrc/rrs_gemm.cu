@@ -4,25 +4,36 @@
 //   P_g[t][n] = sum_{k in group g} qX[t][k] * qW[n][k]          (exact int32)
 //   Y[t][n]   = (sum_g s_g * P_g[t][n]) * scale_t[t] * scale_w[n]
 //
-// The smoothing scale s_g is shared by every element of group g, so it cannot
-// be folded into the integer operands; it is applied group-wise to exact
-// integer partial sums, which is the hardware-aligned scheme the rebuttal page
-// describes ("Novelty": reorder, then a group-wise smoothing scale).
+// The smoothing scale s_g is shared by all elements of group g and is a
+// runtime float, so it cannot be folded into the integer operands; it is
+// applied group-wise to exact integer partial sums -- the hardware-aligned
+// scheme the rebuttal page describes ("Novelty": reorder, then a group-wise
+// smoothing scale).
 //
-// Kernel structure (one CTA per 128 x BN output tile, 13 warps):
-//   warps 0-7   epilogue: per group, tcgen05.ld the int32 partial from TMEM,
-//               convert exactly, acc += s_g * P_g in fp32 registers; at the
-//               end Y = acc * scale_t * scale_w.
-//   warps 8-11  producers: load packed INT4 rows of qX / qW, unpack to INT8
-//               (sign-correct by placing each nibble in the high half of a
-//               byte, i.e. 16 * q), store into the 128-byte-swizzled K-major
-//               shared-memory layout the MMA reads.
-//   warp 12     TMEM allocation and, on one thread, tcgen05.mma.kind::i8
-//               (M = 128, N = BN, K = 32 per instruction, 4 per 128-wide K
-//               block) into a double-buffered TMEM accumulator, one buffer per
-//               group.
-// The products are 256 * qX * qW; the partial is shifted right by 8 (exact)
-// before the fp32 conversion.
+// Persistent kernel, one CTA per SM, 128 x 192 output tiles, 16 warps:
+//   warp 0       TMA: int8 activation tile (128 rows x 128 k, 128-byte swizzle)
+//                and packed INT4 weight tile (192 rows x 64 bytes) per k-block
+//   warp 1       tcgen05.mma.kind::i8 (M=128, N=192, K=32, 4 per k-block) into
+//                a double-buffered TMEM accumulator, one buffer per group
+//   warps 2-3    TMEM allocation (warp 2, 512 columns), then unpack the weight
+//                tile to int8 (16 * q, sign-correct without extension) in the
+//                128-byte-swizzled K-major layout
+//   warps 4-15   epilogue, 64 accumulator columns per thread: per group, read
+//                the int32 partial from TMEM, convert it exactly,
+//                acc += s_g * P_g (fp32, packed f32x2); per tile,
+//                Y = acc * scale_t * scale_w
+//
+// Exact int32 -> fp32 without a conversion instruction: every TMEM accumulator
+// starts at the bit pattern of 1.5 * 2^23 (the epilogue writes it back after
+// each read), so after the integer MMAs its bits read as the float
+// 1.5 * 2^23 + 16 * P_g exactly (|16 P_g| < 2^22), and one fp32 subtraction
+// recovers 16 * P_g.  Partials longer than 2048 k are promoted in 2048-wide
+// blocks with the same s_g.
+//
+// k order: inside each 32-wide k chunk both operands store the codes in the
+// order 0,2,4,6,1,3,5,7, 8,10,... (what a nibble mask produces); the integer
+// sum over the chunk does not depend on the order.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -31,94 +42,114 @@
 #include "rrs_internal.h"
 
 namespace rrs {
-
 namespace gemm {
 
 constexpr int BM = 128;
-constexpr int BK = 128;                 // K elements per pipeline stage
-constexpr int NSTAGE = 4;
-constexpr int EPI_WARPS = 8;
-constexpr int PROD_WARPS = 4;
-constexpr int MMA_WARP = EPI_WARPS + PROD_WARPS;
-constexpr int NTHREADS = (MMA_WARP + 1) * 32;
-constexpr int MAX_GROUPS = 256;         // K / G with K <= 32768, G >= 128
-
-template <int BN>
-struct Smem {
-    static constexpr int A_BYTES = BM * BK;         // int8
-    static constexpr int B_BYTES = BN * BK;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES;
-    static constexpr int TOTAL = BAR_OFF + 1024 + MAX_GROUPS * 4 + 1024;   // + alignment slack
-};
+constexpr int BN = 192;
+constexpr int TMEM_BUF = 256;                 // column stride of the two TMEM buffers
+constexpr int BK = 128;
+constexpr int NS = 4;                         // MMA stages (A int8 + B int8)
+constexpr int NP = 4;                         // packed-weight stages
+constexpr int A_BYTES = BM * BK;              // 16 KB
+constexpr int B8_BYTES = BN * BK;             // 24 KB
+constexpr int BP_BYTES = BN * BK / 2;         // 12 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B8 = OFF_A + NS * A_BYTES;
+constexpr int OFF_BP = OFF_B8 + NS * B8_BYTES;
+constexpr int OFF_BAR = OFF_BP + NP * BP_BYTES;
+constexpr int OFF_S = OFF_BAR + 1024;
+constexpr int MAX_PB = 2048;                  // longest promoted block of k
+constexpr int MAX_NPB = 32768 / 128;          // promotion blocks per tile (K <= 32768)
+constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
+constexpr int NTHREADS = 512;
+constexpr int UNPACK_WARPS = 2;
+constexpr int EPI_WARPS = 12;
+constexpr uint32_t kBiasBits = 0x4B400000u;   // 1.5 * 2^23
+constexpr float kBias = 12582912.0f;
 
 struct Args {
-    const uint8_t* qX;
-    const uint8_t* qW;
     const float* s;
     const float* scale_t;
     const float* scale_w;
-    int M, N, K, G;
+    int M, N, K, G, PB;
     float* Y;
-    int32_t* P;
+    int32_t* P;          // debug partials [K/G, M, N] or null
     uint32_t* err;
     uint64_t limit_ns;
 };
 
-// Byte offset of 16-byte logical chunk `lc` of operand row `row` inside a
-// K-major, 128-byte-swizzled tile (8-row atoms of 1024 bytes).
 __device__ __forceinline__ uint32_t sw128_off(int row, int lc) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((lc ^ (row & 7)) << 4));
 }
 
-// 8 packed INT4 codes (reading R9: even k in the low nibble) -> 8 int8 bytes
-// holding 16 * q, in k order.
-__device__ __forceinline__ void unpack8(uint32_t w, uint32_t& o0, uint32_t& o1) {
-    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;   // k = 0, 2, 4, 6 of this word, x16
-    const uint32_t hi = w & 0xF0F0F0F0u;          // k = 1, 3, 5, 7, x16
-    o0 = __byte_perm(lo, hi, 0x5140);             // k 0..3
-    o1 = __byte_perm(lo, hi, 0x7362);             // k 4..7
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
 }
 
-__device__ __forceinline__ void store_unpacked(uint8_t* tile, int row, int pc, uint4 v) {
-    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-    unpack8(v.x, a0, a1);
-    unpack8(v.y, a2, a3);
-    unpack8(v.z, b0, b1);
-    unpack8(v.w, b2, b3);
-    *reinterpret_cast<uint4*>(tile + sw128_off(row, 2 * pc)) = make_uint4(a0, a1, a2, a3);
-    *reinterpret_cast<uint4*>(tile + sw128_off(row, 2 * pc + 1)) = make_uint4(b0, b1, b2, b3);
+__device__ __forceinline__ void arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
 }
 
-template <int BN, bool DEBUG_P>
-__global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(Args g) {
-    using S = Smem<BN>;
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+        "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+template <bool DEBUG_P>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
-    uint64_t* empty = full + NSTAGE;
-    uint64_t* tfull = empty + NSTAGE;
+    uint64_t* afull = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* bfull = afull + NS;
+    uint64_t* mempty = bfull + NS;
+    uint64_t* pfull = mempty + NS;
+    uint64_t* pempty = pfull + NP;
+    uint64_t* tfull = pempty + NP;
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-    float* s_sm = reinterpret_cast<float*>(smem + S::BAR_OFF + 1024);
+    float* s_sm = reinterpret_cast<float*>(smem + OFF_S);
+    volatile int* abortv = abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM;
-    const int n0 = blockIdx.x * BN;
     const int K = g.K;
     const int KB = K / BK;
-    const int NG = K / g.G;
-    const int kb_per_group = g.G / BK;
-    volatile int* abortv = abort_flag;
+    const int NPB = K / g.PB;          // promotion blocks per tile
+    const int kb_per_pb = g.PB / BK;
+    const int nmb = (g.M + BM - 1) / BM;
+    const int nnb = (g.N + BN - 1) / BN;
+    const int ntiles = nmb * nnb;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(&full[i], PROD_WARPS * 32);
-            mbar_init(&empty[i], 1);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&afull[i], 1);
+            mbar_init(&bfull[i], UNPACK_WARPS);
+            mbar_init(&mempty[i], 1);
+        }
+        for (int i = 0; i < NP; ++i) {
+            mbar_init(&pfull[i], 1);
+            mbar_init(&pempty[i], UNPACK_WARPS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
@@ -129,10 +160,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(Args g) {
         mbar_fence_init();
     }
     if (!DEBUG_P) {
-        for (int i = threadIdx.x; i < NG; i += blockDim.x) s_sm[i] = g.s[i];
+        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
     }
-    if (warp == MMA_WARP) {
-        tmem_alloc(tmem_slot, 2 * BN);
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -140,144 +171,201 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(Args g) {
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= EPI_WARPS && warp < MMA_WARP) {
-        // ------------------------------------------------------ producers
-        const int p = threadIdx.x - EPI_WARPS * 32;
-        const int pc = p & 3;
-        const int rsub = p >> 2;
-        const size_t ldk = (size_t)(K / 2);
-        for (int kb = 0; kb < KB; ++kb) {
-            const int slot = kb % NSTAGE;
-            const uint32_t ph = (uint32_t)(kb / NSTAGE) & 1u;
-            uint4 ra[BM / 32];
-            uint4 rb[BN / 32];
-#pragma unroll
-            for (int i = 0; i < BM / 32; ++i) {
-                const int grow = m0 + rsub + 32 * i;
-                ra[i] = grow < g.M ? __ldg(reinterpret_cast<const uint4*>(
-                                         g.qX + (size_t)grow * ldk + (size_t)kb * 64 + pc * 16))
-                                   : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < BN / 32; ++i) {
-                const int grow = n0 + rsub + 32 * i;
-                rb[i] = grow < g.N ? __ldg(reinterpret_cast<const uint4*>(
-                                         g.qW + (size_t)grow * ldk + (size_t)kb * 64 + pc * 16))
-                                   : make_uint4(0, 0, 0, 0);
-            }
-            if (!mbar_wait_bounded(&empty[slot], ph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns))
-                break;
-            uint8_t* at = smem + slot * S::STAGE_BYTES;
-            uint8_t* bt = at + S::A_BYTES;
-#pragma unroll
-            for (int i = 0; i < BM / 32; ++i) store_unpacked(at, rsub + 32 * i, pc, ra[i]);
-#pragma unroll
-            for (int i = 0; i < BN / 32; ++i) store_unpacked(bt, rsub + 32 * i, pc, rb[i]);
-            fence_proxy_async_smem();
-            mbar_arrive(&full[slot]);
-        }
-    } else if (warp == MMA_WARP) {
-        // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(BM, BN);
+    if (warp < 4) {
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- TMA
+            uint32_t it = 0;
             bool ok = true;
-            for (int kb = 0; kb < KB && ok; ++kb) {
-                const int slot = kb % NSTAGE;
-                const uint32_t ph = (uint32_t)(kb / NSTAGE) & 1u;
-                const int gi = kb / kb_per_group;
-                const bool first = (kb % kb_per_group) == 0;
-                const bool last = (kb % kb_per_group) == kb_per_group - 1;
-                const int buf = gi & 1;
-                if (first) {
-                    ok = mbar_wait_bounded(&tempty[buf], (((uint32_t)gi >> 1) & 1u) ^ 1u, abortv,
-                                           g.err, kErrGemmTimeout, g.limit_ns);
-                    if (!ok) break;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % nmb) * BM;
+                const int n0 = (tile / nmb) * BN;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int ps = it % NP;
+                    const uint32_t pph = (it / NP) & 1u;
+                    if (!(ok = mbar_wait_bounded(&pempty[ps], pph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    arrive_expect_tx(&pfull[ps], BP_BYTES);
+                    tma_load_2d(smem + OFF_BP + ps * BP_BYTES, &tmB, kb * (BK / 2), n0, &pfull[ps]);
+                    const int ms = it % NS;
+                    const uint32_t mph = (it / NS) & 1u;
+                    if (!(ok = mbar_wait_bounded(&mempty[ms], mph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    arrive_expect_tx(&afull[ms], A_BYTES);
+                    tma_load_2d(smem + OFF_A + ms * A_BYTES, &tmA, kb * BK, m0, &afull[ms]);
                 }
-                ok = mbar_wait_bounded(&full[slot], ph, abortv, g.err, kErrGemmTimeout, g.limit_ns);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + slot * S::STAGE_BYTES);
-                const uint32_t b_base = a_base + S::A_BYTES;
-                const uint32_t d = tmem + (uint32_t)(buf * BN);
-#pragma unroll
-                for (int k = 0; k < BK / 32; ++k) {
-                    umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc,
-                            (first && k == 0) ? 0u : 1u);
-                }
-                tc_commit(&empty[slot]);
-                if (last) tc_commit(&tfull[buf]);
             }
-            // Wait for every issued MMA before TMEM can be released.
+            if (!ok) {
+                // Give up: let every copy already issued land before the CTA exits.
+                volatile int no_abort = 0;
+                for (uint32_t j = it > NP ? it - NP : 0; j < it + 1; ++j)
+                    mbar_wait_bounded(&pfull[j % NP], (j / NP) & 1u, &no_abort, nullptr, 0, g.limit_ns);
+                for (uint32_t j = it > NS ? it - NS : 0; j < it; ++j)
+                    mbar_wait_bounded(&afull[j % NS], (j / NS) & 1u, &no_abort, nullptr, 0, g.limit_ns);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------------------- MMA
+            constexpr uint32_t idesc = idesc_i8(BM, BN);
+            uint32_t it = 0, gc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const bool first = (kb % kb_per_pb) == 0;
+                    const bool last = (kb % kb_per_pb) == kb_per_pb - 1;
+                    const int buf = gc & 1;
+                    if (first && !(ok = mbar_wait_bounded(&tempty[buf], (gc >> 1) & 1u, abortv, g.err,
+                                                         kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    const int ms = it % NS;
+                    const uint32_t mph = (it / NS) & 1u;
+                    if (!(ok = mbar_wait_bounded(&afull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    if (!(ok = mbar_wait_bounded(&bfull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + OFF_A + ms * A_BYTES);
+                    const uint32_t b_base = smem_u32(smem + OFF_B8 + ms * B8_BYTES);
+                    const uint32_t d = tmem + (uint32_t)(buf * TMEM_BUF);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)
+                        umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc, 1u);
+                    tc_commit(&mempty[ms]);
+                    if (last) {
+                        tc_commit(&tfull[buf]);
+                        ++gc;
+                    }
+                }
+            }
             tc_commit(done);
-            volatile int dummy_abort = 0;
-            mbar_wait_bounded(done, 0, &dummy_abort, g.err, kErrGemmTimeout, g.limit_ns);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
+        } else if (warp >= 2) {
+            // -------------------------------------------------------- unpack
+            const int p = threadIdx.x - 64;            // 0..63
+            const int pc = p & 3;
+            const int r0 = p >> 2;                     // 0..15
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int ps = it % NP;
+                    const uint32_t pph = (it / NP) & 1u;
+                    const int ms = it % NS;
+                    const uint32_t mph = (it / NS) & 1u;
+                    if (!(ok = mbar_wait_bounded(&pfull[ps], pph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    if (!(ok = mbar_wait_bounded(&mempty[ms], mph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    const unsigned char* src = smem + OFF_BP + ps * BP_BYTES;
+                    unsigned char* dst = smem + OFF_B8 + ms * B8_BYTES;
+#pragma unroll 4
+                    for (int j = 0; j < BN / 16; ++j) {
+                        const int row = r0 + 16 * j;
+                        const uint4 v = *reinterpret_cast<const uint4*>(src + row * 64 + pc * 16);
+                        // low nibbles (even k) and high nibbles (odd k), each as 16 * q
+                        const uint4 o0 = make_uint4((v.x << 4) & 0xF0F0F0F0u, v.x & 0xF0F0F0F0u,
+                                                    (v.y << 4) & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u);
+                        const uint4 o1 = make_uint4((v.z << 4) & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                                    (v.w << 4) & 0xF0F0F0F0u, v.w & 0xF0F0F0F0u);
+                        *reinterpret_cast<uint4*>(dst + sw128_off(row, 2 * pc)) = o0;
+                        *reinterpret_cast<uint4*>(dst + sw128_off(row, 2 * pc + 1)) = o1;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&bfull[ms]);
+                        mbar_arrive(&pempty[ps]);
+                    }
+                }
+            }
         }
     } else {
-        // ------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int colhalf = warp >> 2;
-        const int row = m0 + 32 * quarter + lane;
-        const int col0 = n0 + 64 * colhalf;
-        float acc[64];
+        const int cgrp = (warp - 4) >> 2;             // 0..2: 64-column slice of the tile
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+        const int col0 = 64 * cgrp;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) tmem_st32_const(lane_base + b * TMEM_BUF + col0 + 32 * c, kBiasBits);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&tempty[0]);
+            mbar_arrive(&tempty[1]);
+        }
+        const float2 negb = make_float2(-kBias, -kBias);
+        const float2 sixteenth = make_float2(0.0625f, 0.0625f);
+        uint32_t gc = 0;
         bool ok = true;
-        for (int gi = 0; gi < NG; ++gi) {
-            const int buf = gi & 1;
-            ok = mbar_wait_bounded(&tfull[buf], ((uint32_t)gi >> 1) & 1u, abortv, g.err,
-                                   kErrGemmTimeout, g.limit_ns);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(buf * BN + 64 * colhalf);
-            const float sg = DEBUG_P ? 0.0f : s_sm[gi];
+        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            const int m0 = (tile % nmb) * BM;
+            const int n0 = (tile / nmb) * BN;
+            float2 acc[32];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t r[32];
-                tmem_ld32(taddr + 32 * h, r);
-                tmem_ld_wait();
-                if (h == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[buf]);
+            for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            const int row = m0 + 32 * quarter + lane;
+            for (int pb = 0; pb < NPB; ++pb, ++gc) {
+                const int buf = gc & 1;
+                if (!(ok = mbar_wait_bounded(&tfull[buf], (gc >> 1) & 1u, abortv, g.err, kErrGemmTimeout,
+                                             g.limit_ns)))
+                    break;
+                tc_fence_after();
+                const float sg = DEBUG_P ? 0.0f : s_sm[pb];
+                const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[16];
+                    tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 f = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        const float2 p16 = __fadd2_rn(f, negb);            // 16 * P, exact
+                        if (DEBUG_P) acc[8 * c + i] = __ffma2_rn(p16, sixteenth, acc[8 * c + i]);  // exact ints
+                        else acc[8 * c + i] = __ffma2_rn(s2, p16, acc[8 * c + i]);
+                    }
                 }
-                if (DEBUG_P) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) tmem_st32_const(lane_base + buf * TMEM_BUF + col0 + 32 * c, kBiasBits);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                if (DEBUG_P && ((pb + 1) * g.PB) % g.G == 0) {
+                    const int gi = ((pb + 1) * g.PB) / g.G - 1;
                     if (row < g.M) {
                         int32_t* dst = g.P + ((size_t)gi * g.M + row) * g.N;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const int col = col0 + 32 * h + i;
-                            if (col < g.N) dst[col] = ((int32_t)r[i]) >> 8;
+                            const int col = n0 + col0 + 2 * i;
+                            if (col < g.N) dst[col] = (int32_t)acc[i].x;
+                            if (col + 1 < g.N) dst[col + 1] = (int32_t)acc[i].y;
                         }
                     }
-                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float pf = (float)(((int32_t)r[i]) >> 8);
-                        acc[32 * h + i] = __fmaf_rn(sg, pf, acc[32 * h + i]);
-                    }
+                    for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
                 }
             }
-        }
-        if (!DEBUG_P && ok && row < g.M) {
-            const float st = g.scale_t[row];
-            float* yrow = g.Y + (size_t)row * g.N;
-            const bool vec = ((g.N & 3) == 0);
+            if (!DEBUG_P && ok) {
+                // lane l holds scale_w of columns col0 + 2l, 2l + 1; broadcast by shuffles
+                const int cl = n0 + col0 + 2 * lane;
+                const float2 swl = make_float2(cl < g.N ? g.scale_w[cl] : 0.0f, cl + 1 < g.N ? g.scale_w[cl + 1] : 0.0f);
+                const float st = row < g.M ? g.scale_t[row] : 0.0f;
+                const float2 st2 = make_float2(st, st);
+                float* yrow = g.Y + (size_t)row * g.N;
+                const bool vec = (g.N & 1) == 0;
 #pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-                const int col = col0 + i;
-                if (vec && col + 3 < g.N) {
-                    const float4 sw = __ldg(reinterpret_cast<const float4*>(g.scale_w + col));
-                    float4 y;
-                    y.x = __fmul_rn(__fmul_rn(acc[i], st), sw.x);
-                    y.y = __fmul_rn(__fmul_rn(acc[i + 1], st), sw.y);
-                    y.z = __fmul_rn(__fmul_rn(acc[i + 2], st), sw.z);
-                    y.w = __fmul_rn(__fmul_rn(acc[i + 3], st), sw.w);
-                    *reinterpret_cast<float4*>(yrow + col) = y;
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (col + u < g.N)
-                            yrow[col + u] = __fmul_rn(__fmul_rn(acc[i + u], st), g.scale_w[col + u]);
+                for (int i = 0; i < 32; ++i) {
+                    const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i), __shfl_sync(0xffffffffu, swl.y, i));
+                    const int col = n0 + col0 + 2 * i;
+                    const float2 y = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
+                    if (row < g.M) {
+                        if (vec && col + 1 < g.N) {
+                            *reinterpret_cast<float2*>(yrow + col) = y;
+                        } else {
+                            if (col < g.N) yrow[col] = y.x;
+                            if (col + 1 < g.N) yrow[col + 1] = y.y;
+                        }
+                    }
                 }
             }
         }
@@ -285,9 +373,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(Args g) {
 
     tc_fence_before();
     __syncthreads();
-    if (warp == MMA_WARP) {
+    if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * BN);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -307,14 +395,47 @@ __global__ void wait_probe_kernel(uint64_t limit_ns, uint32_t* err) {
     }
 }
 
+// ------------------------------------------------------------------ host ---
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+static bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gemm
 
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
-    constexpr int BN = 128;
-    using S = gemm::Smem<BN>;
-    gemm::Args a;
-    a.qX = gl.qX;
-    a.qW = gl.qW;
+    using namespace gemm;
+    CUtensorMap tmA, tmB;
+    if (!make_map_u8(&tmA, gl.qX8, (uint64_t)gl.K, (uint64_t)gl.M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K / 2, (uint64_t)gl.N, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    Args a;
     a.s = gl.s;
     a.scale_t = gl.scale_t;
     a.scale_w = gl.scale_w;
@@ -322,22 +443,27 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     a.N = gl.N;
     a.K = gl.K;
     a.G = gl.G;
+    a.PB = gl.G < MAX_PB ? gl.G : MAX_PB;
     a.Y = gl.Y;
     a.P = gl.P;
     a.err = gl.err;
     a.limit_ns = kWaitLimitNs;
-    dim3 grid((gl.N + BN - 1) / BN, (gl.M + gemm::BM - 1) / gemm::BM);
-    const int smem = S::TOTAL;
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int ntiles = ((gl.M + BM - 1) / BM) * ((gl.N + BN - 1) / BN);
+    const int grid = ntiles < nsm ? ntiles : nsm;
+    cudaError_t e;
     if (gl.P) {
-        auto kern = gemm::gemm_kernel<BN, true>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        auto kern = gemm_kernel<true>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
-        kern<<<grid, gemm::NTHREADS, smem, stream>>>(a);
+        kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
     } else {
-        auto kern = gemm::gemm_kernel<BN, false>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        auto kern = gemm_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
-        kern<<<grid, gemm::NTHREADS, smem, stream>>>(a);
+        kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
     }
     return cudaGetLastError();
 }

@@ -26,9 +26,9 @@ struct PrepLaunch {
 cudaError_t launch_prep(const PrepLaunch& pl, cudaStream_t stream);
 
 struct GemmLaunch {
-    const uint8_t* qX;      // [M, K/2]
-    const uint8_t* qW;      // [N, K/2]
-    const float* s;         // [K/G] (null = all ones)
+    const int8_t* qX8;      // [M, K] int8 activation codes (k order of the fast prep / expand kernels)
+    const uint8_t* qW;      // [N, K/2] packed INT4 weights
+    const float* s;         // [K/G]
     const float* scale_t;   // [M]
     const float* scale_w;   // [N]
     int M, N, K, G;
@@ -37,7 +37,30 @@ struct GemmLaunch {
     uint32_t* err;          // workspace error word
 };
 
+// Fast activation path (K % 2048 == 0): rotation + reorder + group max into an
+// fp32 scratch, then smoothing + quantisation.
+struct PrepFastLaunch {
+    const void* X;          // fp16 [rows, K]
+    int rows, K, n, G;
+    float c_n;
+    const int32_t* perm;
+    int unit_scales;
+    float* s;               // [K/G] output (max of |X'| per group, or 1)
+    uint8_t* qX;            // [rows, K/2]
+    int8_t* qX8;            // [rows, K]
+    float* scale_t;         // [rows]
+    float* scratch;         // [rows, K] fp32
+};
+
+bool prep_fast_supported(int K, int n);
+size_t prep_fast_scratch_bytes(int M, int K);
+cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t stream);
+// Packed INT4 rows -> int8 rows in the GEMM's k order.
+cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStream_t stream);
+
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream);
+cudaError_t launch_divide_check(const float* a, const float* b, int n, float* q_fast, float* q_ieee,
+                                cudaStream_t stream);
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, uint32_t* err, cudaStream_t stream);
 

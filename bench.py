@@ -153,7 +153,8 @@ def run_ours(args):
                              ws=st["ws"])
             if events is not None:
                 events[j][1].record(stream)
-            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW"], st["sw"], L.G, Y=st["Y"], ws=st["ws"])
+            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW"], st["sw"], L.G, Y=st["Y"], ws=st["ws"],
+                          flags=rrs.WS_HOLDS_A8)
             if events is not None:
                 events[j][2].record(stream)
 
@@ -233,7 +234,7 @@ def run_ours(args):
     prep_bytes = [2 * st["L"].M * st["L"].K + st["L"].M * st["L"].K // 2 + 4 * st["L"].M + 4 * (st["L"].K // st["L"].G)
                   for st in state]
     prep_gbs = sum(prep_bytes) / (sum(prep_ms) * 1e-3) / 1e9
-    launches_per_step = 3 * len(state)      # group-max, quantise, GEMM per layer
+    launches_per_step = 3 * len(state)      # rotate+group max, smooth+quantise, GEMM per layer
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,

@@ -85,10 +85,16 @@ typedef enum {
 /* flags */
 #define RRS_NO_ROTATE 1u         /* identity instead of the Hadamard (plain Runtime Smooth) */
 #define RRS_FORCE_UNIT_SCALES 2u /* s := 1 for every group (A4W4 per-channel scheme, no smoothing) */
+#define RRS_WS_HOLDS_A8 4u       /* rrs_w4a4_gemm: the workspace already holds the int8 activation
+                                    operand that rrs_smooth_quant wrote for this qX (same ws, same
+                                    stream, nothing in between); skips re-expanding qX */
 
-/* Bytes of workspace the calls below need for this problem (>= 256).  The
- * workspace must be zero-filled once before first use; it holds the kernels'
- * error word and any split-K scratch. */
+/* Bytes of workspace the calls below need for this problem.  Layout: a
+ * 256-byte header holding the kernels' error word (zero-fill it once before
+ * first use), then the int8 copy of the activation codes that the GEMM's
+ * tensor cores read (M*K bytes), then, when K is a multiple of 2048, the
+ * reordered fp32 activations X' that pass between the two activation kernels
+ * (M*K*4 bytes).  rrs_w4a4_gemm alone needs only the first two parts. */
 size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags);
 
 /* Offline weight path (summary page "Approach"; rebuttal page "Description of
@@ -109,10 +115,12 @@ rrs_status rrs_smooth_quant(const void *X, int M, int K, int G, int had_block, c
 
 /* Group-scaled W4A4 GEMM (rebuttal page "Novelty": the smoothing scale is
  * applied group-wise to match the hardware GEMM): exact int32 P_g per group
- * on the tensor cores, Y = (sum_g s_g * P_g) * scale_t * scale_w in fp32. */
+ * on the tensor cores, Y = (sum_g s_g * P_g) * scale_t * scale_w in fp32.
+ * flags: 0, or RRS_WS_HOLDS_A8 (see above).  Without it the packed qX is
+ * first expanded into the workspace's int8 operand. */
 rrs_status rrs_w4a4_gemm(const uint8_t *qX, const float *s, const float *scale_t, const uint8_t *qW,
                          const float *scale_w, int M, int N, int K, int G, float *Y, void *ws,
-                         size_t ws_bytes, rrs_stream_t stream);
+                         size_t ws_bytes, unsigned flags, rrs_stream_t stream);
 
 /* rrs_smooth_quant followed by rrs_w4a4_gemm on one stream, no host sync.
  * qX, s and scale_t are caller-provided intermediate buffers. */
@@ -156,6 +164,13 @@ rrs_status rrs_check_workspace(void *ws, rrs_stream_t stream);
  * microseconds (1..1000000).  The kernel records the timeout in the
  * workspace error word and returns; the context stays usable. */
 rrs_status rrs_debug_wait_timeout(int limit_us, void *ws, size_t ws_bytes, rrs_stream_t stream);
+
+/* Self-test hook for tests: q_fast[i] = a[i] / b[i] computed the way the
+ * activation kernels divide (Markstein's correction from the correctly
+ * rounded reciprocal of b, for b > 0), q_ieee[i] = the IEEE fp32 division.
+ * All device arrays of length n. */
+rrs_status rrs_debug_divide(const float *a, const float *b, int n, float *q_fast, float *q_ieee,
+                            rrs_stream_t stream);
 
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char *rrs_last_error_string(void);

@@ -80,12 +80,15 @@ def test_argument_checks_fail_before_any_launch(L):
     assert L.rrs_prepare_weights(ok, 16, 384, 256, ok, ok, ok, 0, None) == 1
     ws = ok
     # G not dividing K -> invalid; G not a multiple of 128 -> unsupported
-    assert L.rrs_smooth_quant(ok, 16, 256, 100, 256, ok, ok, ok, ok, ws, 256, 0, None) == 1
-    assert L.rrs_smooth_quant(ok, 16, 256, 64, 256, ok, ok, ok, ok, ws, 256, 0, None) == 2
+    assert L.rrs_smooth_quant(ok, 16, 256, 100, 256, ok, ok, ok, ok, ws, 1 << 20, 0, None) == 1
+    assert L.rrs_smooth_quant(ok, 16, 256, 64, 256, ok, ok, ok, ok, ws, 1 << 20, 0, None) == 2
     # workspace too small
     assert L.rrs_smooth_quant(ok, 16, 256, 128, 256, ok, ok, ok, ok, ws, 8, 0, None) == 5
+    need = L.rrs_workspace_size(16, 16, 4096, 128, 4096, 0)
+    assert need >= 256 + 16 * 4096 + 16 * 4096 * 4
+    assert L.rrs_smooth_quant(ok, 16, 4096, 128, 4096, ok, ok, ok, ok, ws, need - 1, 0, None) == 5
     # M < 1
-    assert L.rrs_w4a4_gemm(ok, ok, ok, ok, ok, 0, 16, 256, 128, ok, ws, 256, None) == 1
+    assert L.rrs_w4a4_gemm(ok, ok, ok, ok, ok, 0, 16, 256, 128, ok, ws, 1 << 20, 0, None) == 1
     assert L.rrs_debug_wait_timeout(0, ws, 256, None) == 1
     assert len(L.rrs_last_error_string()) > 0
 

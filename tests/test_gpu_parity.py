@@ -247,3 +247,38 @@ def test_bounded_wait_reports_timeout_and_context_survives(rrs):
     assert e.value.status_name == "RRS_ERR_TIMEOUT"
     rrs.check_workspace(ws)                     # cleared
     test_tiny_full_parity(rrs, "identity")      # the context still works
+
+
+def test_markstein_division_matches_ieee(rrs):
+    """The activation kernels divide with Markstein's correction from RN(1/b);
+    over the divisions they perform (|a| <= 8 b, b > 0) it must equal the IEEE
+    quotient.  Hard cases: every divisor mantissa pattern class, quotients next
+    to representable ties, exact multiples, tiny numerators."""
+    rng = np.random.default_rng(123)
+    n = 1 << 22
+    e = rng.integers(-40, 40, size=n)
+    mant = rng.integers(0, 1 << 23, size=n)
+    mant[: n // 16] = (1 << 23) - 1                      # all-ones mantissas
+    mant[n // 16: n // 8] = 0                            # powers of two
+    mant[n // 8: n // 8 + n // 16] = rng.integers((1 << 23) - 64, 1 << 23, size=n // 16)
+    b = np.ldexp(1.0 + mant / 2.0 ** 23, e).astype(np.float32)
+    k = rng.uniform(-8.0, 8.0, size=n)
+    a = (k * b.astype(np.float64)).astype(np.float32)
+    q = rng.integers(-8, 8, size=n).astype(np.float32)     # exact multiples and their neighbours
+    sel = slice(n // 4, n // 2)
+    a[sel] = (q[sel] * b[sel]).astype(np.float32)
+    ulp_steps = rng.integers(-3, 4, size=n).astype(np.int32)
+    sel2 = slice(n // 2, 3 * n // 4)
+    a[sel2] = (a[sel2].view(np.int32) + ulp_steps[sel2]).view(np.float32)
+    a[3 * n // 4: 3 * n // 4 + 1024] = 0.0
+    tiny = slice(7 * n // 8, n)
+    a[tiny] = (b[tiny].astype(np.float64) * rng.uniform(-1, 1, size=n // 8) * 2.0 ** -30).astype(np.float32)
+    ad = torch.from_numpy(a).to(DEV)
+    bd = torch.from_numpy(b).to(DEV)
+    qf, qi = rrs.debug_divide(ad, bd)
+    qf, qi = qf.cpu().numpy(), qi.cpu().numpy()
+    same = (qf.view(np.uint32) == qi.view(np.uint32)) | ((qf == 0) & (qi == 0))
+    assert same.all(), f"{np.count_nonzero(~same)} quotients differ, e.g. a={a[~same][:3]} b={b[~same][:3]}"
+    # and the IEEE division itself is the correctly rounded quotient (checked in double)
+    ref = (a.astype(np.float64) / b.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(qi, ref)
