@@ -46,11 +46,27 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// Tests phase completion; if the phase is still open the warp is suspended
+// (issuing nothing) until it completes or about `hint_ns` pass, so waiting
+// warps do not steal issue slots from working warps on the same scheduler.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns = 20000u) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of phase completion.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -61,15 +77,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity of `bar` has completed.  Gives
 // up after `limit_ns`, or as soon as another thread of the CTA has raised
 // *abort; on giving up it records `err_bit` in the workspace error word, raises
-// *abort and returns false.
+// *abort and returns false.  SPIN polls without suspending (lowest hand-off
+// latency, for the few single-thread and producer roles); otherwise the warp
+// sleeps in try_wait between polls.
+template <bool SPIN = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, uint32_t* err,
                                                   uint32_t err_bit, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (SPIN ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (SPIN ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if ((it & (SPIN ? 1023u : 3u)) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 if (err) atomicOr(err, err_bit);

@@ -11,8 +11,9 @@
 // smoothing scale).
 //
 // Persistent kernel, one CTA per SM, 128 x 192 output tiles, 16 warps:
-//   warp 0       TMA: int8 activation tile (128 rows x 128 k, 128-byte swizzle)
-//                and packed INT4 weight tile (192 rows x 64 bytes) per k-block
+//   warp 0       TMA, one thread driving two independent streams: packed INT4
+//                weight tiles (192 rows x 64 bytes) and int8 activation tiles
+//                (128 rows x 128 k, 128-byte swizzle) per k-block
 //   warp 1       tcgen05.mma.kind::i8 (M=128, N=192, K=32, 4 per k-block) into
 //                a double-buffered TMEM accumulator, one buffer per group
 //   warps 2-3    TMEM allocation (warp 2, 512 columns), then unpack the weight
@@ -23,11 +24,10 @@
 //                acc += s_g * P_g (fp32, packed f32x2); per tile,
 //                Y = acc * scale_t * scale_w
 //
-// Exact int32 -> fp32 without a conversion instruction: every TMEM accumulator
-// starts at the bit pattern of 1.5 * 2^23 (the epilogue writes it back after
-// each read), so after the integer MMAs its bits read as the float
-// 1.5 * 2^23 + 16 * P_g exactly (|16 P_g| < 2^22), and one fp32 subtraction
-// recovers 16 * P_g.  Partials longer than 2048 k are promoted in 2048-wide
+// Exact int32 -> fp32 without a conversion instruction: adding the bit pattern
+// of 1.5 * 2^23 to the int32 partial 16 * P_g gives the bits of the float
+// 1.5 * 2^23 + 16 * P_g exactly (|16 P_g| <= 2^22), and one fp32 subtraction
+// recovers 16 * P_g (exact for |16 P_g| <= 2^22, i.e. groups of up to 4096 k).  Longer groups are promoted in 4096-wide
 // blocks with the same s_g.
 //
 // k order: inside each 32-wide k chunk both operands store the codes in the
@@ -49,7 +49,7 @@ constexpr int BN = 192;
 constexpr int TMEM_BUF = 256;                 // column stride of the two TMEM buffers
 constexpr int BK = 128;
 constexpr int NS = 4;                         // MMA stages (A int8 + B int8)
-constexpr int NP = 4;                         // packed-weight stages
+constexpr int NP = 5;                         // packed-weight stages
 constexpr int A_BYTES = BM * BK;              // 16 KB
 constexpr int B8_BYTES = BN * BK;             // 24 KB
 constexpr int BP_BYTES = BN * BK / 2;         // 12 KB
@@ -58,7 +58,7 @@ constexpr int OFF_B8 = OFF_A + NS * A_BYTES;
 constexpr int OFF_BP = OFF_B8 + NS * B8_BYTES;
 constexpr int OFF_BAR = OFF_BP + NP * BP_BYTES;
 constexpr int OFF_S = OFF_BAR + 1024;
-constexpr int MAX_PB = 2048;                  // longest promoted block of k
+constexpr int MAX_PB = 4096;                  // longest promoted block of k (|16 P| <= 2^22 stays exact)
 constexpr int MAX_NPB = 32768 / 128;          // promotion blocks per tile (K <= 32768)
 constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
 constexpr int NTHREADS = 512;
@@ -174,33 +174,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp < 4) {
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- TMA
-            uint32_t it = 0;
+            // One thread, two independent streams: packed weight tiles (bounded
+            // only by the unpack freeing a slot) and activation tiles (bounded by
+            // the MMA freeing a stage).  Neither waits behind the other.
+            const uint32_t my_tiles = blockIdx.x < (unsigned)ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+            const uint32_t total = my_tiles * KB;
+            uint32_t itB = 0, itA = 0;
+            uint64_t t0 = 0;
+            uint32_t idle = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                const int m0 = (tile % nmb) * BM;
-                const int n0 = (tile / nmb) * BN;
-                for (int kb = 0; kb < KB; ++kb, ++it) {
-                    const int ps = it % NP;
-                    const uint32_t pph = (it / NP) & 1u;
-                    if (!(ok = mbar_wait_bounded(&pempty[ps], pph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
-                        break;
+            while (itB < total || itA < total) {
+                bool progress = false;
+                if (itB < total && mbar_test_wait(&pempty[itB % NP], ((itB / NP) & 1u) ^ 1u)) {
+                    const int tile = blockIdx.x + (itB / KB) * gridDim.x;
+                    const int ps = itB % NP;
                     arrive_expect_tx(&pfull[ps], BP_BYTES);
-                    tma_load_2d(smem + OFF_BP + ps * BP_BYTES, &tmB, kb * (BK / 2), n0, &pfull[ps]);
-                    const int ms = it % NS;
-                    const uint32_t mph = (it / NS) & 1u;
-                    if (!(ok = mbar_wait_bounded(&mempty[ms], mph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
-                        break;
+                    tma_load_2d(smem + OFF_BP + ps * BP_BYTES, &tmB, (itB % KB) * (BK / 2), (tile / nmb) * BN,
+                                &pfull[ps]);
+                    ++itB;
+                    progress = true;
+                }
+                if (itA < total && mbar_test_wait(&mempty[itA % NS], ((itA / NS) & 1u) ^ 1u)) {
+                    const int tile = blockIdx.x + (itA / KB) * gridDim.x;
+                    const int ms = itA % NS;
                     arrive_expect_tx(&afull[ms], A_BYTES);
-                    tma_load_2d(smem + OFF_A + ms * A_BYTES, &tmA, kb * BK, m0, &afull[ms]);
+                    tma_load_2d(smem + OFF_A + ms * A_BYTES, &tmA, (itA % KB) * BK, (tile % nmb) * BM, &afull[ms]);
+                    ++itA;
+                    progress = true;
+                }
+                if (progress) {
+                    idle = 0;
+                    continue;
+                }
+                // bounded wait: give up after the limit or when another role gave up
+                if (idle++ == 0) t0 = globaltimer_ns();
+                if ((idle & 1023u) == 0) {
+                    if (*abortv) { ok = false; break; }
+                    if (globaltimer_ns() - t0 > g.limit_ns) {
+                        atomicOr(g.err, kErrGemmTimeout);
+                        *abortv = 1;
+                        ok = false;
+                        break;
+                    }
                 }
             }
             if (!ok) {
-                // Give up: let every copy already issued land before the CTA exits.
+                // let every copy already issued land before the CTA exits
                 volatile int no_abort = 0;
-                for (uint32_t j = it > NP ? it - NP : 0; j < it + 1; ++j)
-                    mbar_wait_bounded(&pfull[j % NP], (j / NP) & 1u, &no_abort, nullptr, 0, g.limit_ns);
-                for (uint32_t j = it > NS ? it - NS : 0; j < it; ++j)
-                    mbar_wait_bounded(&afull[j % NS], (j / NS) & 1u, &no_abort, nullptr, 0, g.limit_ns);
+                for (uint32_t j = itB > NP ? itB - NP : 0; j < itB; ++j)
+                    mbar_wait_bounded<true>(&pfull[j % NP], (j / NP) & 1u, &no_abort, nullptr, 0, g.limit_ns);
+                for (uint32_t j = itA > NS ? itA - NS : 0; j < itA; ++j)
+                    mbar_wait_bounded<true>(&afull[j % NS], (j / NS) & 1u, &no_abort, nullptr, 0, g.limit_ns);
             }
         } else if (warp == 1 && lane == 0) {
             // -------------------------------------------------------- MMA
@@ -212,20 +236,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const bool first = (kb % kb_per_pb) == 0;
                     const bool last = (kb % kb_per_pb) == kb_per_pb - 1;
                     const int buf = gc & 1;
-                    if (first && !(ok = mbar_wait_bounded(&tempty[buf], (gc >> 1) & 1u, abortv, g.err,
+                    if (first && !(ok = mbar_wait_bounded<true>(&tempty[buf], (gc >> 1) & 1u, abortv, g.err,
                                                          kErrGemmTimeout, g.limit_ns)))
                         break;
                     const int ms = it % NS;
                     const uint32_t mph = (it / NS) & 1u;
-                    if (!(ok = mbar_wait_bounded(&afull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
-                    if (!(ok = mbar_wait_bounded(&bfull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    if (!(ok = mbar_wait_bounded<true>(&afull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    if (!(ok = mbar_wait_bounded<true>(&bfull[ms], mph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + OFF_A + ms * A_BYTES);
                     const uint32_t b_base = smem_u32(smem + OFF_B8 + ms * B8_BYTES);
                     const uint32_t d = tmem + (uint32_t)(buf * TMEM_BUF);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k)
-                        umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc, 1u);
+                        umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc,
+                                (first && k == 0) ? 0u : 1u);
                     tc_commit(&mempty[ms]);
                     if (last) {
                         tc_commit(&tfull[buf]);
@@ -249,20 +274,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t pph = (it / NP) & 1u;
                     const int ms = it % NS;
                     const uint32_t mph = (it / NS) & 1u;
-                    if (!(ok = mbar_wait_bounded(&pfull[ps], pph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
-                    if (!(ok = mbar_wait_bounded(&mempty[ms], mph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
+                    if (!(ok = mbar_wait_bounded<true>(&pfull[ps], pph, abortv, g.err, kErrGemmTimeout, g.limit_ns))) break;
+                    if (!(ok = mbar_wait_bounded<true>(&mempty[ms], mph ^ 1u, abortv, g.err, kErrGemmTimeout, g.limit_ns)))
                         break;
                     const unsigned char* src = smem + OFF_BP + ps * BP_BYTES;
                     unsigned char* dst = smem + OFF_B8 + ms * B8_BYTES;
-#pragma unroll 4
+                    // All loads first, then all stores: the compiler cannot move a
+                    // shared load above a shared store it cannot prove disjoint.
+                    uint4 v[BN / 16];
+#pragma unroll
+                    for (int j = 0; j < BN / 16; ++j)
+                        v[j] = *reinterpret_cast<const uint4*>(src + (r0 + 16 * j) * 64 + pc * 16);
+#pragma unroll
                     for (int j = 0; j < BN / 16; ++j) {
                         const int row = r0 + 16 * j;
-                        const uint4 v = *reinterpret_cast<const uint4*>(src + row * 64 + pc * 16);
                         // low nibbles (even k) and high nibbles (odd k), each as 16 * q
-                        const uint4 o0 = make_uint4((v.x << 4) & 0xF0F0F0F0u, v.x & 0xF0F0F0F0u,
-                                                    (v.y << 4) & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u);
-                        const uint4 o1 = make_uint4((v.z << 4) & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
-                                                    (v.w << 4) & 0xF0F0F0F0u, v.w & 0xF0F0F0F0u);
+                        const uint4 o0 = make_uint4((v[j].x << 4) & 0xF0F0F0F0u, v[j].x & 0xF0F0F0F0u,
+                                                    (v[j].y << 4) & 0xF0F0F0F0u, v[j].y & 0xF0F0F0F0u);
+                        const uint4 o1 = make_uint4((v[j].z << 4) & 0xF0F0F0F0u, v[j].z & 0xF0F0F0F0u,
+                                                    (v[j].w << 4) & 0xF0F0F0F0u, v[j].w & 0xF0F0F0F0u);
                         *reinterpret_cast<uint4*>(dst + sw128_off(row, 2 * pc)) = o0;
                         *reinterpret_cast<uint4*>(dst + sw128_off(row, 2 * pc + 1)) = o1;
                     }
@@ -281,14 +311,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int cgrp = (warp - 4) >> 2;             // 0..2: 64-column slice of the tile
         const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
         const int col0 = 64 * cgrp;
-#pragma unroll
-        for (int b = 0; b < 2; ++b)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) tmem_st32_const(lane_base + b * TMEM_BUF + col0 + 32 * c, kBiasBits);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
+        if (lane == 0) {                      // both accumulator buffers start free
             mbar_arrive(&tempty[0]);
             mbar_arrive(&tempty[1]);
         }
@@ -312,24 +335,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const float sg = DEBUG_P ? 0.0f : s_sm[pb];
                 const float2 s2 = make_float2(sg, sg);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[16];
+                for (int c = 0; c < 4; c += 2) {
+                    uint32_t r[16], r2[16];
                     tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c, r);
+                    tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c + 16, r2);
                     tmem_ld_wait();
+                    if (c == 2) {
+                        // all of this warp's columns are in registers: release the buffer
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[buf]);
+                    }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float2 f = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                        const float2 p16 = __fadd2_rn(f, negb);            // 16 * P, exact
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t* rr = i < 8 ? r : r2;
+                        const int ii = i & 7;
+                        // bits of 1.5 * 2^23 + 16 P as a float, minus 1.5 * 2^23: exact 16 P
+                        const float2 f = make_float2(__uint_as_float(rr[2 * ii] + kBiasBits),
+                                                     __uint_as_float(rr[2 * ii + 1] + kBiasBits));
+                        const float2 p16 = __fadd2_rn(f, negb);
                         if (DEBUG_P) acc[8 * c + i] = __ffma2_rn(p16, sixteenth, acc[8 * c + i]);  // exact ints
                         else acc[8 * c + i] = __ffma2_rn(s2, p16, acc[8 * c + i]);
                     }
                 }
-#pragma unroll
-                for (int c = 0; c < 2; ++c) tmem_st32_const(lane_base + buf * TMEM_BUF + col0 + 32 * c, kBiasBits);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
                 if (DEBUG_P && ((pb + 1) * g.PB) % g.G == 0) {
                     const int gi = ((pb + 1) * g.PB) / g.G - 1;
                     if (row < g.M) {

@@ -136,12 +136,24 @@ __global__ void __launch_bounds__(MAXT) rot_gather_kernel(RotArgs p) {
                      (size_t)team * 2 * K;
     const int bar_id = 1 + team;
 
-    // gather addresses of this thread's outputs j in [64t, 64t + 64) (one group)
+    // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
+    // perm is staged through shared memory: coalesced 16-byte global loads, and
+    // 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
+    // chunk reads below are bank-conflict free.
     uint32_t gaddr[32];
+    {
+        int4* pst = reinterpret_cast<int4*>(smem_raw);
+        const int4* pg = reinterpret_cast<const int4*>(p.perm);
+        for (int c = threadIdx.x; c < K / 4; c += blockDim.x) pst[c ^ ((c >> 4) & 7)] = pg[c];
+        __syncthreads();
 #pragma unroll
-    for (int l = 0; l < E; l += 2) {
-        const int j = t * E + l;
-        gaddr[l / 2] = (uint32_t)swz(p.perm[j]) | ((uint32_t)swz(p.perm[j + 1]) << 16);
+        for (int m = 0; m < 16; ++m) {
+            const int c = t * 16 + m;
+            const int4 v = pst[c ^ ((c >> 4) & 7)];
+            gaddr[2 * m] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
+            gaddr[2 * m + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
+        }
+        __syncthreads();   // the row buffers reuse this space
     }
     float tmax = 0.0f;
 
