@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <numeric>
 #include <vector>
 
@@ -172,6 +173,42 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
     return RRS_OK;
 }
 
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Scratch for rrs_smooth_quant_noalloc: a fixed device array, so that the call
+// needs no workspace from the caller.  Every device that loads this library
+// holds it (about 5 MiB) until the process exits.  In host code the name
+// g_noalloc_ws is only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, once per device.
+namespace {
+constexpr size_t kNoAllocMaxElems = (size_t)1 << 20;   // M * K limit
+constexpr size_t kNoAllocBytes = kHeaderBytes + kNoAllocMaxElems + kNoAllocMaxElems * 4;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_ws[kNoAllocBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_ws on the current device (looked up on first use).
+rrs_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(RRS_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return RRS_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -374,6 +411,38 @@ rrs_status rrs_debug_divide(const float* a, const float* b, int n, float* q_fast
     cudaError_t e = rrs::launch_divide_check(a, b, n, q_fast, q_ieee, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "divide check kernel");
     return RRS_OK;
+}
+
+rrs_status rrs_smooth_quant_noalloc(const void* X, int M, int K, int G, int had_block, const int32_t* perm,
+                                    uint8_t* qX, float* s, float* scale_t, unsigned flags, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(X);
+    RRS_REQUIRE_PTR(perm);
+    RRS_REQUIRE_PTR(qX);
+    RRS_REQUIRE_PTR(s);
+    RRS_REQUIRE_PTR(scale_t);
+    if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    const size_t need = ws_bytes_full(M, K, n);
+    if ((size_t)M * (size_t)K > kNoAllocMaxElems || need > kNoAllocBytes)
+        return fail(RRS_ERR_UNSUPPORTED,
+                    "rrs_smooth_quant_noalloc: M*K = %zu exceeds its fixed scratch limit of %zu elements; "
+                    "use rrs_smooth_quant with a workspace",
+                    (size_t)M * (size_t)K, kNoAllocMaxElems);
+    void* ws = nullptr;
+    r = noalloc_scratch(&ws);
+    if (r != RRS_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps the previous call's contents: clear the error word.
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-allocation scratch header)");
+    return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, s, scale_t, ws, flags, st);
 }
 
 const char* rrs_last_error_string(void) { return g_last_error; }

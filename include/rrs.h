@@ -172,6 +172,27 @@ rrs_status rrs_debug_wait_timeout(int limit_us, void *ws, size_t ws_bytes, rrs_s
 rrs_status rrs_debug_divide(const float *a, const float *b, int n, float *q_fast, float *q_ieee,
                             rrs_stream_t stream);
 
+/* rrs_smooth_quant without a workspace argument, for callers that cannot
+ * allocate device memory at call time: code running under an allocator it
+ * does not own (a host framework or inference server that hands out only the
+ * tensors it manages), code that must not allocate on its latency-critical
+ * path, or code that cannot know a workspace size in advance.  There is no
+ * counterpart on the pages; it computes exactly what rrs_smooth_quant
+ * computes, with the same outputs and the same limits, plus one more:
+ * M * K <= 1048576 (RRS_ERR_UNSUPPORTED above that).
+ * The scratch is one fixed array in device memory that every GPU which loads
+ * the library holds (about 5 MiB) until the process exits; this function calls
+ * no cudaMalloc, cudaFree or allocating library routine.  The first call on a
+ * device looks up that device's address of the array (cudaGetSymbolAddress,
+ * with the device current), so make the first call on each device before any
+ * stream capture.  All calls share the array: calls whose work overlaps on the
+ * GPU (different streams, or different host threads without ordering) race on
+ * it and must be serialised by the caller.  Each call clears the array's
+ * error word; kernel timeouts are not reported through this entry point. */
+rrs_status rrs_smooth_quant_noalloc(const void *X, int M, int K, int G, int had_block,
+                                    const int32_t *perm, uint8_t *qX, float *s, float *scale_t,
+                                    unsigned flags, rrs_stream_t stream);
+
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char *rrs_last_error_string(void);
 
