@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "librrs.so")
 NO_ROTATE = 1
 FORCE_UNIT_SCALES = 2
 WS_HOLDS_A8 = 4
+W_EXPANDED = 8
 
 _STATUS = {
     0: "RRS_OK",
@@ -57,7 +58,8 @@ def lib() -> ctypes.CDLL:
         "rrs_w4a4_gemm": ([P, P, P, P, P, I, I, I, I, P, P, Z, U, P], I),
         "rrs_linear": ([P, P, P, P, I, I, I, I, I, P, P, P, P, P, Z, U, P], I),
         "rrs_linear_from_host": ([P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, Z, U, P], I),
-        "rrs_w4a4_gemm_debug_partials": ([P, P, I, I, I, I, P, P, Z, P], I),
+        "rrs_w4a4_gemm_debug_partials": ([P, P, I, I, I, I, P, P, Z, U, P], I),
+        "rrs_expand_weights": ([P, I, I, P, P], I),
         "rrs_channel_absmax": ([P, I, I, I, P, U, P], I),
         "rrs_perm_from_channel_max": ([P, I, P], I),
         "rrs_check_workspace": ([P, P], I),
@@ -147,16 +149,24 @@ def smooth_quant(X: torch.Tensor, perm: torch.Tensor, G: int, had_block: int, fl
     return qX, s, scale_t
 
 
+def _need_weights(qW: torch.Tensor, N: int, K: int, flags: int):
+    if flags & W_EXPANDED:
+        _need(qW, "qW", torch.int8, (N, K))
+    else:
+        _need(qW, "qW", torch.uint8, (N, K // 2))
+
+
 def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torch.Tensor,
               scale_w: torch.Tensor, G: int, Y: Optional[torch.Tensor] = None,
               ws: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
     """Group-scaled W4A4 GEMM -> Y fp32 [M, N].  flags=WS_HOLDS_A8 when ``ws`` is the
-    workspace the preceding smooth_quant of this qX wrote (skips re-expanding qX)."""
+    workspace the preceding smooth_quant of this qX wrote (skips re-expanding qX);
+    W_EXPANDED when ``qW`` is the int8 operand from expand_weights."""
     M, K2 = qX.shape
     N = qW.shape[0]
     K = 2 * K2
     _need(qX, "qX", torch.uint8, (M, K2))
-    _need(qW, "qW", torch.uint8, (N, K2))
+    _need_weights(qW, N, K, flags)
     _need(s, "s", torch.float32, (K // G,))
     _need(scale_t, "scale_t", torch.float32, (M,))
     _need(scale_w, "scale_w", torch.float32, (N,))
@@ -178,7 +188,7 @@ def linear(X: torch.Tensor, qW: torch.Tensor, scale_w: torch.Tensor, perm: torch
     N = qW.shape[0]
     dev = X.device
     _need(X, "X", torch.float16, (M, K))
-    _need(qW, "qW", torch.uint8, (N, K // 2))
+    _need_weights(qW, N, K, flags)
     _need(scale_w, "scale_w", torch.float32, (N,))
     _need(perm, "perm", torch.int32, (K,))
     qX = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if qX is None else qX
@@ -214,19 +224,31 @@ def linear_from_host(X_host: torch.Tensor, X_dev: torch.Tensor, qW: torch.Tensor
 
 
 def w4a4_gemm_debug_partials(qX: torch.Tensor, qW: torch.Tensor, G: int, P: Optional[torch.Tensor] = None,
-                             ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                             ws: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
     """Exact per-group int32 partial sums P [K/G, M, N] (debug, small problems)."""
     M, K2 = qX.shape
     N = qW.shape[0]
     K = 2 * K2
     _need(qX, "qX", torch.uint8, (M, K2))
-    _need(qW, "qW", torch.uint8, (N, K2))
+    _need_weights(qW, N, K, flags)
     P = torch.empty((K // G, M, N), dtype=torch.int32, device=qX.device) if P is None else P
     _need(P, "P", torch.int32, (K // G, M, N))
     ws = make_workspace(M, N, K, G, 1, 0, qX.device) if ws is None else ws
     _check(lib().rrs_w4a4_gemm_debug_partials(_ptr(qX), _ptr(qW), M, N, K, G, _ptr(P), _ptr(ws), ws.numel(),
-                                              _stream(stream)))
+                                              flags & W_EXPANDED, _stream(stream)))
     return P
+
+
+def expand_weights(qW: torch.Tensor, qW8: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Int8 tensor-core operand [N, K] (16 q, GEMM k order) from packed INT4 weights [N, K/2];
+    pass it with flags=W_EXPANDED."""
+    N, K2 = qW.shape
+    K = 2 * K2
+    _need(qW, "qW", torch.uint8, (N, K2))
+    qW8 = torch.empty((N, K), dtype=torch.int8, device=qW.device) if qW8 is None else qW8
+    _need(qW8, "qW8", torch.int8, (N, K))
+    _check(lib().rrs_expand_weights(_ptr(qW), N, K, _ptr(qW8), _stream(stream)))
+    return qW8
 
 
 def channel_absmax(X: torch.Tensor, had_block: int, flags: int = 0, cmax: Optional[torch.Tensor] = None,

@@ -168,6 +168,7 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
     gl.Y = Y;
     gl.P = P;
     gl.err = reinterpret_cast<uint32_t*>(ws);
+    gl.w_expanded = (flags & RRS_W_EXPANDED) != 0;
     cudaError_t e = rrs::launch_gemm(gl, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM kernel");
     return RRS_OK;
@@ -299,7 +300,8 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
                       size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
-    return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes, RRS_WS_HOLDS_A8, stream);
+    return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes,
+                         RRS_WS_HOLDS_A8 | (flags & RRS_W_EXPANDED), stream);
 }
 
 rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* qW, const float* scale_w,
@@ -324,7 +326,8 @@ rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* 
 }
 
 rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, int M, int N, int K, int G,
-                                        int32_t* P, void* ws, size_t ws_bytes, rrs_stream_t stream) {
+                                        int32_t* P, void* ws, size_t ws_bytes, unsigned flags,
+                                        rrs_stream_t stream) {
     RRS_REQUIRE_PTR(qX);
     RRS_REQUIRE_PTR(qW);
     RRS_REQUIRE_PTR(P);
@@ -335,8 +338,19 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, in
     if (r != RRS_OK) return r;
     r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
-    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws, 0u,
-                               reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws,
+                               flags & RRS_W_EXPANDED, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, int8_t* qW8, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(qW);
+    RRS_REQUIRE_PTR(qW8);
+    if (N < 1) return fail(RRS_ERR_INVALID_ARG, "N = %d", N);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    cudaError_t e = rrs::launch_expand_weights(qW, qW8, N, K, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "expand_weights kernel");
+    return RRS_OK;
 }
 
 rrs_status rrs_channel_absmax(const void* X, int M, int K, int had_block, float* cmax, unsigned flags,

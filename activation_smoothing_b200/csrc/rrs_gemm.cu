@@ -112,6 +112,107 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Epilogue warps (4 .. 15): per promotion block, read the int32 partial
+// sums of this warp's 32 rows x 64 columns from TMEM, promote them exactly to
+// fp32 and accumulate s_g * P_g; at the end of a tile apply scale_t * scale_w
+// and store Y (or, in debug mode, store the exact per-group partials).
+template <bool DEBUG_P>
+__device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint64_t* tfull, uint64_t* tempty,
+                                              const float* s_sm, volatile int* abortv, int warp, int lane,
+                                              int ntiles, int nmb, int NPB) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int cgrp = (warp - 4) >> 2;             // 0..2: 64-column slice of the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int col0 = 64 * cgrp;
+    if (lane == 0) {                      // both accumulator buffers start free
+        mbar_arrive(&tempty[0]);
+        mbar_arrive(&tempty[1]);
+    }
+    const float2 negb = make_float2(-kBias, -kBias);
+    const float2 sixteenth = make_float2(0.0625f, 0.0625f);
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % nmb) * BM;
+        const int n0 = (tile / nmb) * BN;
+        float2 acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        const int row = m0 + 32 * quarter + lane;
+        for (int pb = 0; pb < NPB; ++pb, ++gc) {
+            const int buf = gc & 1;
+            if (!(ok = mbar_wait_bounded(&tfull[buf], (gc >> 1) & 1u, abortv, g.err, kErrGemmTimeout,
+                                         g.limit_ns)))
+                break;
+            tc_fence_after();
+            const float sg = DEBUG_P ? 0.0f : s_sm[pb];
+            const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t r[16], r2[16];
+                tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c, r);
+                tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c + 16, r2);
+                tmem_ld_wait();
+                if (c == 2) {
+                    // all of this warp's columns are in registers: release the buffer
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t* rr = i < 8 ? r : r2;
+                    const int ii = i & 7;
+                    // bits of 1.5 * 2^23 + 16 P as a float, minus 1.5 * 2^23: exact 16 P
+                    const float2 f = make_float2(__uint_as_float(rr[2 * ii] + kBiasBits),
+                                                 __uint_as_float(rr[2 * ii + 1] + kBiasBits));
+                    const float2 p16 = __fadd2_rn(f, negb);
+                    if (DEBUG_P) acc[8 * c + i] = __ffma2_rn(p16, sixteenth, acc[8 * c + i]);  // exact ints
+                    else acc[8 * c + i] = __ffma2_rn(s2, p16, acc[8 * c + i]);
+                }
+            }
+            if (DEBUG_P && ((pb + 1) * g.PB) % g.G == 0) {
+                const int gi = ((pb + 1) * g.PB) / g.G - 1;
+                if (row < g.M) {
+                    int32_t* dst = g.P + ((size_t)gi * g.M + row) * g.N;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int col = n0 + col0 + 2 * i;
+                        if (col < g.N) dst[col] = (int32_t)acc[i].x;
+                        if (col + 1 < g.N) dst[col + 1] = (int32_t)acc[i].y;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            }
+        }
+        if (!DEBUG_P && ok) {
+            // lane l holds scale_w of columns col0 + 2l, 2l + 1; broadcast by shuffles
+            const int cl = n0 + col0 + 2 * lane;
+            const float2 swl = make_float2(cl < g.N ? g.scale_w[cl] : 0.0f, cl + 1 < g.N ? g.scale_w[cl + 1] : 0.0f);
+            const float st = row < g.M ? g.scale_t[row] : 0.0f;
+            const float2 st2 = make_float2(st, st);
+            float* yrow = g.Y + (size_t)row * g.N;
+            const bool vec = (g.N & 1) == 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i), __shfl_sync(0xffffffffu, swl.y, i));
+                const int col = n0 + col0 + 2 * i;
+                const float2 y = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
+                if (row < g.M) {
+                    if (vec && col + 1 < g.N) {
+                        *reinterpret_cast<float2*>(yrow + col) = y;
+                    } else {
+                        if (col < g.N) yrow[col] = y.x;
+                        if (col + 1 < g.N) yrow[col + 1] = y.y;
+                    }
+                }
+            }
+        }
+    }
+}
+
 template <bool DEBUG_P>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
@@ -306,99 +407,161 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int quarter = warp & 3;
-        const int cgrp = (warp - 4) >> 2;             // 0..2: 64-column slice of the tile
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
-        const int col0 = 64 * cgrp;
-        if (lane == 0) {                      // both accumulator buffers start free
-            mbar_arrive(&tempty[0]);
-            mbar_arrive(&tempty[1]);
-        }
-        const float2 negb = make_float2(-kBias, -kBias);
-        const float2 sixteenth = make_float2(0.0625f, 0.0625f);
-        uint32_t gc = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-            const int m0 = (tile % nmb) * BM;
-            const int n0 = (tile / nmb) * BN;
-            float2 acc[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            const int row = m0 + 32 * quarter + lane;
-            for (int pb = 0; pb < NPB; ++pb, ++gc) {
-                const int buf = gc & 1;
-                if (!(ok = mbar_wait_bounded(&tfull[buf], (gc >> 1) & 1u, abortv, g.err, kErrGemmTimeout,
-                                             g.limit_ns)))
-                    break;
-                tc_fence_after();
-                const float sg = DEBUG_P ? 0.0f : s_sm[pb];
-                const float2 s2 = make_float2(sg, sg);
-#pragma unroll
-                for (int c = 0; c < 4; c += 2) {
-                    uint32_t r[16], r2[16];
-                    tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c, r);
-                    tmem_ld16(lane_base + buf * TMEM_BUF + col0 + 16 * c + 16, r2);
-                    tmem_ld_wait();
-                    if (c == 2) {
-                        // all of this warp's columns are in registers: release the buffer
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[buf]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t* rr = i < 8 ? r : r2;
-                        const int ii = i & 7;
-                        // bits of 1.5 * 2^23 + 16 P as a float, minus 1.5 * 2^23: exact 16 P
-                        const float2 f = make_float2(__uint_as_float(rr[2 * ii] + kBiasBits),
-                                                     __uint_as_float(rr[2 * ii + 1] + kBiasBits));
-                        const float2 p16 = __fadd2_rn(f, negb);
-                        if (DEBUG_P) acc[8 * c + i] = __ffma2_rn(p16, sixteenth, acc[8 * c + i]);  // exact ints
-                        else acc[8 * c + i] = __ffma2_rn(s2, p16, acc[8 * c + i]);
-                    }
-                }
-                if (DEBUG_P && ((pb + 1) * g.PB) % g.G == 0) {
-                    const int gi = ((pb + 1) * g.PB) / g.G - 1;
-                    if (row < g.M) {
-                        int32_t* dst = g.P + ((size_t)gi * g.M + row) * g.N;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int col = n0 + col0 + 2 * i;
-                            if (col < g.N) dst[col] = (int32_t)acc[i].x;
-                            if (col + 1 < g.N) dst[col + 1] = (int32_t)acc[i].y;
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
-                }
-            }
-            if (!DEBUG_P && ok) {
-                // lane l holds scale_w of columns col0 + 2l, 2l + 1; broadcast by shuffles
-                const int cl = n0 + col0 + 2 * lane;
-                const float2 swl = make_float2(cl < g.N ? g.scale_w[cl] : 0.0f, cl + 1 < g.N ? g.scale_w[cl + 1] : 0.0f);
-                const float st = row < g.M ? g.scale_t[row] : 0.0f;
-                const float2 st2 = make_float2(st, st);
-                float* yrow = g.Y + (size_t)row * g.N;
-                const bool vec = (g.N & 1) == 0;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i), __shfl_sync(0xffffffffu, swl.y, i));
-                    const int col = n0 + col0 + 2 * i;
-                    const float2 y = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
-                    if (row < g.M) {
-                        if (vec && col + 1 < g.N) {
-                            *reinterpret_cast<float2*>(yrow + col) = y;
-                        } else {
-                            if (col < g.N) yrow[col] = y.x;
-                            if (col + 1 < g.N) yrow[col + 1] = y.y;
-                        }
-                    }
-                }
-            }
-        }
+        epilogue_role<DEBUG_P>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
     }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
 
+// ------------------------------------------------------------------------
+// Variant for weights stored as the expanded int8 operand (16 q in the GEMM's
+// k order, written once by rrs_expand_weights).  Nothing is unpacked, so the
+// CTA needs no unpack warps; warps 0, 2 and 3 instead each feed the stage ring.
+// A bulk copy's round trip is not overlapped with the next copy a warp issues,
+// so one producer warp keeps one stage in flight and three keep three: stage
+// `it` is loaded by producer it % 3, its activation tile and weight tile by
+// lanes 0 and 1 of that warp in one instruction, onto one barrier.
+namespace w8 {
+constexpr int NST = 5;                        // stages of activation + weight tiles (40 KB each)
+constexpr int NPROD = 3;                      // producer warps
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + NST * A_BYTES;
+constexpr int OFF_BAR = OFF_B + NST * B8_BYTES;
+constexpr int OFF_S = OFF_BAR + 1024;
+constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
+static_assert(SMEM <= 227 * 1024, "shared memory budget");
+static_assert(OFF_B % 1024 == 0 && B8_BYTES % 1024 == 0, "128-byte-swizzled tiles need 1024-byte alignment");
+}  // namespace w8
+
+template <bool DEBUG_P>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + w8::OFF_BAR);
+    uint64_t* empty = full + w8::NST;
+    uint64_t* tfull = empty + w8::NST;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    float* s_sm = reinterpret_cast<float*>(smem + w8::OFF_S);
+    volatile int* abortv = abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int KB = g.K / BK;
+    const int NPB = g.K / g.PB;
+    const int kb_per_pb = g.PB / BK;
+    const int nmb = (g.M + BM - 1) / BM;
+    const int nnb = (g.N + BN - 1) / BN;
+    const int ntiles = nmb * nnb;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < w8::NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], EPI_WARPS);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (!DEBUG_P) {
+        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 || warp == 2 || warp == 3) {
+        // -------------------------------------------------------- TMA
+        const uint32_t p = warp == 0 ? 0u : (uint32_t)(warp - 1);
+        const uint32_t my_tiles = blockIdx.x < (unsigned)ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        const uint32_t total = my_tiles * KB;
+        uint32_t last = 0xFFFFFFFFu;          // last stage this warp loaded
+        bool ok = true;
+        for (uint32_t it = p; it < total; it += w8::NPROD) {
+            const int st = (int)(it % w8::NST);
+            uint32_t free = 1;
+            if (lane == 0)
+                free = mbar_wait_bounded<true>(&empty[st], ((it / w8::NST) & 1u) ^ 1u, abortv, g.err, kErrGemmTimeout,
+                                               g.limit_ns) ? 1u : 0u;
+            if (!__shfl_sync(0xffffffffu, free, 0)) {
+                ok = false;
+                break;
+            }
+            const int tile = blockIdx.x + (int)(it / KB) * gridDim.x;
+            const int kb = (int)(it % KB);
+            if (lane == 0) arrive_expect_tx(&full[st], A_BYTES + B8_BYTES);
+            __syncwarp();
+            if (lane < 2) {
+                unsigned char* dst = lane == 0 ? smem + w8::OFF_A + st * A_BYTES : smem + w8::OFF_B + st * B8_BYTES;
+                const CUtensorMap* map = lane == 0 ? &tmA : &tmB;
+                const int y = lane == 0 ? (tile % nmb) * BM : (tile / nmb) * BN;
+                tma_load_2d(dst, map, kb * BK, y, &full[st]);
+            }
+            __syncwarp();
+            last = it;
+        }
+        if (!ok && lane == 0 && last != 0xFFFFFFFFu) {
+            // let this warp's copies land before the CTA exits
+            volatile int no_abort = 0;
+            mbar_wait_bounded<true>(&full[last % w8::NST], (last / w8::NST) & 1u, &no_abort, nullptr, 0, g.limit_ns);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // -------------------------------------------------------- MMA
+            constexpr uint32_t idesc = idesc_i8(BM, BN);
+            uint32_t it = 0, gc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const bool first = (kb % kb_per_pb) == 0;
+                    const bool lastk = (kb % kb_per_pb) == kb_per_pb - 1;
+                    const int buf = gc & 1;
+                    if (first && !(ok = mbar_wait_bounded<true>(&tempty[buf], (gc >> 1) & 1u, abortv, g.err,
+                                                                kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    const int st = (int)(it % w8::NST);
+                    if (!(ok = mbar_wait_bounded<true>(&full[st], (it / w8::NST) & 1u, abortv, g.err,
+                                                       kErrGemmTimeout, g.limit_ns)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + w8::OFF_A + st * A_BYTES);
+                    const uint32_t b_base = smem_u32(smem + w8::OFF_B + st * B8_BYTES);
+                    const uint32_t d = tmem + (uint32_t)(buf * TMEM_BUF);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)
+                        umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc,
+                                (first && k == 0) ? 0u : 1u);
+                    tc_commit(&empty[st]);
+                    if (lastk) {
+                        tc_commit(&tfull[buf]);
+                        ++gc;
+                    }
+                }
+            }
+            tc_commit(done);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
+        }
+    } else {
+        epilogue_role<DEBUG_P>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {
@@ -461,8 +624,13 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     CUtensorMap tmA, tmB;
     if (!make_map_u8(&tmA, gl.qX8, (uint64_t)gl.K, (uint64_t)gl.M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K / 2, (uint64_t)gl.N, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (gl.w_expanded) {
+        if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K, (uint64_t)gl.N, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    } else if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K / 2, (uint64_t)gl.N, BK / 2, BN,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) {
         return cudaErrorInvalidValue;
+    }
     Args a;
     a.s = gl.s;
     a.scale_t = gl.scale_t;
@@ -482,7 +650,12 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     const int ntiles = ((gl.M + BM - 1) / BM) * ((gl.N + BN - 1) / BN);
     const int grid = ntiles < nsm ? ntiles : nsm;
     cudaError_t e;
-    if (gl.P) {
+    if (gl.w_expanded) {
+        auto kern = gl.P ? gemm_w8_kernel<true> : gemm_w8_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w8::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, NTHREADS, w8::SMEM, stream>>>(tmA, tmB, a);
+    } else if (gl.P) {
         auto kern = gemm_kernel<true>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;

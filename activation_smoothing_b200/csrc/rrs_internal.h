@@ -27,7 +27,7 @@ cudaError_t launch_prep(const PrepLaunch& pl, cudaStream_t stream);
 
 struct GemmLaunch {
     const int8_t* qX8;      // [M, K] int8 activation codes (k order of the fast prep / expand kernels)
-    const uint8_t* qW;      // [N, K/2] packed INT4 weights
+    const uint8_t* qW;      // [N, K/2] packed INT4 weights, or [N, K] int8 16 q when w_expanded
     const float* s;         // [K/G]
     const float* scale_t;   // [M]
     const float* scale_w;   // [N]
@@ -35,6 +35,7 @@ struct GemmLaunch {
     float* Y;               // [M, N] (null in debug mode)
     int32_t* P;             // [K/G, M, N] debug partials (null in normal mode)
     uint32_t* err;          // workspace error word
+    bool w_expanded;        // qW holds the expanded operand written by launch_expand_weights
 };
 
 // Fast activation path (K % 2048 == 0): rotation + reorder + group max into an
@@ -57,6 +58,8 @@ size_t prep_fast_scratch_bytes(int M, int K);
 cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t stream);
 // Packed INT4 rows -> int8 rows in the GEMM's k order.
 cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStream_t stream);
+// Packed INT4 weight rows -> int8 rows holding 16 q, in the same k order.
+cudaError_t launch_expand_weights(const uint8_t* qW, int8_t* qW8, int N, int K, cudaStream_t stream);
 
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream);
 cudaError_t launch_divide_check(const float* a, const float* b, int n, float* q_fast, float* q_ieee,

@@ -383,6 +383,16 @@ __global__ void expand_kernel(const uint8_t* qX, int8_t* qX8, size_t nwords) {
     }
 }
 
+// Packed INT4 weight rows -> int8 operand rows holding 16 q (the nibble in
+// the high half of each byte), in the k order of expand_kernel.  The GEMM's
+// epilogue expects the factor 16 on the weight side.
+__global__ void expand_weights_kernel(const uint8_t* qW, int8_t* qW8, size_t nwords) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwords; i += (size_t)gridDim.x * blockDim.x) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(qW)[i];
+        reinterpret_cast<uint2*>(qW8)[i] = make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
+    }
+}
+
 // Self-test of div_markstein against the IEEE division, elementwise.
 __global__ void divide_check_kernel(const float* a, const float* b, int n, float* q_fast, float* q_ieee) {
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -486,6 +496,17 @@ cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStre
     size_t blocks = (nwords + 255) / 256;
     if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
     fast::expand_kernel<<<(unsigned)blocks, 256, 0, st>>>(qX, qX8, nwords);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expand_weights(const uint8_t* qW, int8_t* qW8, int N, int K, cudaStream_t st) {
+    const size_t nwords = (size_t)N * K / 8;
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    size_t blocks = (nwords + 255) / 256;
+    if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
+    fast::expand_weights_kernel<<<(unsigned)blocks, 256, 0, st>>>(qW, qW8, nwords);
     return cudaGetLastError();
 }
 

@@ -88,6 +88,9 @@ typedef enum {
 #define RRS_WS_HOLDS_A8 4u       /* rrs_w4a4_gemm: the workspace already holds the int8 activation
                                     operand that rrs_smooth_quant wrote for this qX (same ws, same
                                     stream, nothing in between); skips re-expanding qX */
+#define RRS_W_EXPANDED 8u        /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host and the debug
+                                    partials: qW points at the int8 operand that rrs_expand_weights
+                                    wrote ([N, K] bytes) instead of the packed INT4 codes */
 
 /* Bytes of workspace the calls below need for this problem.  Layout: a
  * 256-byte header holding the kernels' error word (zero-fill it once before
@@ -142,8 +145,20 @@ rrs_status rrs_linear_from_host(const void *X_host, void *X_dev, const uint8_t *
 /* Debug: the exact per-group partial sums P [K/G, M, N] (int32) of the same
  * GEMM, written instead of Y.  For small problems only. */
 rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t *qX, const uint8_t *qW, int M, int N, int K,
-                                        int G, int32_t *P, void *ws, size_t ws_bytes,
+                                        int G, int32_t *P, void *ws, size_t ws_bytes, unsigned flags,
                                         rrs_stream_t stream);
+
+/* Weight operand for the tensor cores, written once per layer after
+ * rrs_prepare_weights: qW8[n][k'] = 16 * q, where q is the signed INT4 code
+ * that qW packs, laid out in the GEMM's k order (within each 8 codes: the
+ * even k, then the odd k).  The pages have no counterpart: the INT4 codes
+ * themselves are unchanged, only stored one per byte so that the GEMM needs
+ * no unpacking step on the chip.  It doubles the weight bytes (N * K instead
+ * of N * K / 2) and makes the GEMM faster where it is compute-bound (prefill;
+ * pass RRS_W_EXPANDED).  qW packed [N, K/2] as rrs_prepare_weights writes it;
+ * qW8 [N, K] device, caller-owned, 16-byte aligned.  K as for rrs_w4a4_gemm.
+ * Asynchronous on `stream`. */
+rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, int8_t *qW8, rrs_stream_t stream);
 
 /* Calibration statistic for the reorder index: cmax[k] = max_t |X_rot[t][k]|
  * (rotation only, no reorder).  cmax fp32 [K]. */

@@ -46,8 +46,13 @@ def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
     qX, s, st = rrs.smooth_quant(Xd, pd, G, n, flags)
     ws = rrs.make_workspace(X.shape[0], W.shape[0], K, G, n, flags)
     Y = rrs.w4a4_gemm(qX, s, st, qW, sw, G, ws=ws)
+    # the expanded-weight kernel computes the same exact partials and the same
+    # fp32 promotion in the same order: its Y must be bit-identical
+    qW8 = rrs.expand_weights(qW)
+    Y8 = rrs.w4a4_gemm(qX, s, st, qW8, sw, G, ws=ws, flags=rrs.W_EXPANDED)
     rrs.check_workspace(ws)
     torch.cuda.synchronize()
+    assert_bits_equal(Y8, Y, "Y (expanded weights) vs Y (packed weights)")
 
     _, oqX, os_, ost = oracle.smooth_quant(X, G, n_eff, perm.numpy(), unit_scales=unit)
     assert_bits_equal(s, os_, "s")
@@ -89,6 +94,34 @@ def test_tiny_partials_bit_exact(rrs):
     _, oqW, _ = oracle.prepare_weights(W, L.had_block, perm.numpy())
     P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(oqX).to(DEV), torch.from_numpy(oqW).to(DEV), L.G)
     assert_bits_equal(P, oracle.group_partials(oqX, oqW, L.G), "P_g")
+
+
+def expanded_operand(q_packed: np.ndarray) -> np.ndarray:
+    """16 q per byte, k order 0,2,4,6,1,3,5,7 within each 8 codes (from the oracle's packed codes)."""
+    N, K2 = q_packed.shape
+    codes = oracle.unpack(q_packed, 2 * K2).astype(np.int32)          # [N, K] natural k order
+    order = np.array([0, 2, 4, 6, 1, 3, 5, 7])
+    idx = (np.arange(2 * K2).reshape(-1, 8)[:, order]).reshape(-1)
+    return (16 * codes[:, idx]).astype(np.int8)
+
+
+def test_expand_weights_operand_bit_exact(rrs):
+    L = wl.LAYERS["tiny"]
+    W = wl.make_weights(L)
+    perm = wl.random_perm(L.K, 3)
+    _, oqW, _ = oracle.prepare_weights(W, L.had_block, perm.numpy())
+    qW8 = rrs.expand_weights(torch.from_numpy(oqW).to(DEV))
+    assert_bits_equal(qW8, expanded_operand(oqW), "qW8")
+
+
+@pytest.mark.parametrize("M,N,K,G", [(130, 520, 1024, 128), (257, 136, 512, 256)])
+def test_partials_bit_exact_expanded_weights(rrs, M, N, K, G):
+    rng = np.random.default_rng(M + N)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    qW8 = rrs.expand_weights(torch.from_numpy(qW).to(DEV))
+    P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(qX).to(DEV), qW8, G, flags=rrs.W_EXPANDED)
+    assert_bits_equal(P, oracle.group_partials(qX, qW, G), "P_g (expanded weights)")
 
 
 def test_partials_extreme_codes(rrs):
@@ -225,6 +258,14 @@ def test_linear_equals_two_calls_and_host_path(rrs):
     rrs.linear_from_host(Xh, torch.empty_like(Xd), qW, sw, perm, L.G, L.had_block,
                          torch.empty_like(qX), torch.empty_like(s), torch.empty_like(st),
                          torch.empty((M, N), dtype=torch.float32, device=DEV), Yh, ws)
+    assert torch.equal(Yh, Y1.cpu())
+    qW8 = rrs.expand_weights(qW)
+    Y3 = rrs.linear(Xd, qW8, sw, perm, L.G, L.had_block, flags=rrs.W_EXPANDED)
+    rrs.linear_from_host(Xh, torch.empty_like(Xd), qW8, sw, perm, L.G, L.had_block,
+                         torch.empty_like(qX), torch.empty_like(s), torch.empty_like(st),
+                         torch.empty((M, N), dtype=torch.float32, device=DEV), Yh, ws, flags=rrs.W_EXPANDED)
+    torch.cuda.synchronize()
+    assert torch.equal(Y3, Y1)
     assert torch.equal(Yh, Y1.cpu())
 
 
