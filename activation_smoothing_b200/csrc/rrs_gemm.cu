@@ -194,18 +194,34 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
             const float st = row < g.M ? g.scale_t[row] : 0.0f;
             const float2 st2 = make_float2(st, st);
             float* yrow = g.Y + (size_t)row * g.N;
-            const bool vec = (g.N & 1) == 0;
+            // Each lane owns one row, so a warp's store touches 32 rows.  Whole
+            // 32-byte sectors per lane (8 columns, one 256-bit store) keep the
+            // L2 from merging partial sectors; ragged edges, N % 8 != 0 and a Y
+            // not 32-byte aligned fall back to scalar stores.
+            const bool v8 = (g.N & 7) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 31u) == 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i), __shfl_sync(0xffffffffu, swl.y, i));
-                const int col = n0 + col0 + 2 * i;
-                const float2 y = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
+            for (int j = 0; j < 8; ++j) {
+                float2 y[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = 4 * j + q;
+                    const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i),
+                                                  __shfl_sync(0xffffffffu, swl.y, i));
+                    y[q] = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
+                }
+                const int col = n0 + col0 + 8 * j;
                 if (row < g.M) {
-                    if (vec && col + 1 < g.N) {
-                        *reinterpret_cast<float2*>(yrow + col) = y;
+                    if (v8 && col + 7 < g.N) {
+                        asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                                     ::"l"(yrow + col), "f"(y[0].x), "f"(y[0].y), "f"(y[1].x), "f"(y[1].y),
+                                       "f"(y[2].x), "f"(y[2].y), "f"(y[3].x), "f"(y[3].y)
+                                     : "memory");
                     } else {
-                        if (col < g.N) yrow[col] = y.x;
-                        if (col + 1 < g.N) yrow[col + 1] = y.y;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (col + 2 * q < g.N) yrow[col + 2 * q] = y[q].x;
+                            if (col + 2 * q + 1 < g.N) yrow[col + 2 * q + 1] = y[q].y;
+                        }
                     }
                 }
             }

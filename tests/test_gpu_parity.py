@@ -124,6 +124,26 @@ def test_partials_bit_exact_expanded_weights(rrs, M, N, K, G):
     assert_bits_equal(P, oracle.group_partials(qX, qW, G), "P_g (expanded weights)")
 
 
+@pytest.mark.parametrize("M,N", [(130, 520), (67, 200)])
+def test_y_not_32_byte_aligned_matches(rrs, M, N):
+    """A Y that is 16- but not 32-byte aligned takes the scalar store path: same values."""
+    K, G = 512, 128
+    rng = np.random.default_rng(M)
+    qX = torch.from_numpy(rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)).to(DEV)
+    qW = torch.from_numpy(rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)).to(DEV)
+    s = torch.rand(K // G, device=DEV) + 0.5
+    st = torch.rand(M, device=DEV)
+    sw = torch.rand(N, device=DEV)
+    Y = rrs.w4a4_gemm(qX, s, st, qW, sw, G)
+    big = torch.zeros(M * N + 8, dtype=torch.float32, device=DEV)
+    Yoff = big[4:4 + M * N].view(M, N)
+    assert Yoff.data_ptr() % 32 == 16
+    rrs.w4a4_gemm(qX, s, st, qW, sw, G, Y=Yoff)
+    torch.cuda.synchronize()
+    assert_bits_equal(Yoff, Y, "Y at a 16-byte offset")
+    assert torch.all(big[:4] == 0) and torch.all(big[4 + M * N:] == 0)
+
+
 def test_partials_extreme_codes(rrs):
     """All codes -8 or 7 (|P_g| at its maximum 64 G) stay exact."""
     rng = np.random.default_rng(1)
