@@ -30,9 +30,11 @@ sys.path.insert(0, ROOT)
 METRIC = "RRS W4A4 linear TOPS (prep+GEMM) at LLaMA-3-8B shapes; % of INT8 TC peak"
 UNIT = "TOPS"
 N_XSETS = 4            # distinct activation buffers per layer, rotated between steps
-# DRAM bytes per GEMM launch from the ncu capture in profiles/ (None until measured
-# for the current kernel).
-GEMM_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) per GEMM launch, mean over the q/o, k/v and gate/up
+# launches of one step, from the ncu capture summarised in
+# profiles/gemm_kernel_llama3_8b.md.  Must go back to None whenever gemm_kernel
+# changes until it is captured again.
+GEMM_TRAFFIC_BYTES = 44.4e6
 
 
 def peaks():
@@ -130,9 +132,10 @@ def run_ours(args):
         perm = rrs.calibrate_perm(Xc, L.had_block)
         W = wl.make_weights(L).to(dev)
         qW, sw = rrs.prepare_weights(W, perm, L.had_block)
+        qW8 = rrs.expand_weights(qW)          # secondary path: weights one code per byte
         del W
         xs = [wl.make_activations(L, sample=2 + i + 10 * rank).to(dev) for i in range(N_XSETS)]
-        st = dict(L=L, perm=perm, qW=qW, sw=sw, xs=xs,
+        st = dict(L=L, perm=perm, qW=qW, qW8=qW8, sw=sw, xs=xs,
                   qX=torch.empty((L.M, L.K // 2), dtype=torch.uint8, device=dev),
                   s=torch.empty(L.K // L.G, dtype=torch.float32, device=dev),
                   st=torch.empty(L.M, dtype=torch.float32, device=dev),
@@ -194,6 +197,44 @@ def run_ours(args):
     ops_step = sum(st["L"].ops for st in state)
     value = ops_step * K * world / (ms * 1e-3) / 1e12
 
+    # ---- secondary: the same step with the weights expanded offline to the int8
+    # operand (rrs_expand_weights + RRS_W_EXPANDED); same codes, same results.
+    Kx = max(3, min(K, 500))
+    xg = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in state]
+
+    def step_expanded(i, timed):
+        for j, st in enumerate(state):
+            L = st["L"]
+            rrs.smooth_quant(st["xs"][i % N_XSETS], st["perm"], L.G, L.had_block, qX=st["qX"], s=st["s"],
+                             scale_t=st["st"], ws=st["ws"])
+            if timed:
+                xg[j][0].record(stream)
+            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW8"], st["sw"], L.G, Y=st["Y"], ws=st["ws"],
+                          flags=rrs.WS_HOLDS_A8 | rrs.W_EXPANDED)
+            if timed:
+                xg[j][1].record(stream)
+    for i in range(3):
+        step_expanded(i, False)
+    torch.cuda.synchronize()
+    xa, xb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    xa.record(stream)
+    for i in range(Kx):
+        step_expanded(i, True)
+    xb.record(stream)
+    torch.cuda.synchronize()
+    # per-layer GEMM times from the last step's events (all steps are alike)
+    xgemm = [xg[j][0].elapsed_time(xg[j][1]) for j in range(len(state))]
+    xms = xa.elapsed_time(xb)
+    if pg:
+        t = torch.tensor([xms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        xms = float(t.item())
+    for st in state:
+        rrs.check_workspace(st["ws"])
+    expanded = {"value": round(ops_step * Kx * world / (xms * 1e-3) / 1e12, 2), "unit": UNIT, "steps": Kx,
+                "gemm_ms_per_layer_last_step": [round(x, 5) for x in xgemm],
+                "weights": "INT4 codes stored one per byte as 16 q (rrs_expand_weights); 2x weight bytes"}
+
     # ---- end to end through the C ABI with host buffers (pinned), copies timed.
     e2e = None
     if not args.no_e2e:
@@ -240,7 +281,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 MMA / fp32 prep",
-        "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights)",
+        "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights); weights packed INT4",
         "config": {"workload": "+".join(names),
                    "shapes": [dict(M=st["L"].M, K=st["L"].K, N=st["L"].N, G=st["L"].G, had=st["L"].had_block)
                               for st in state],
@@ -248,11 +289,13 @@ def run_ours(args):
                    "l2": f"activations rotate over {N_XSETS} sets per layer; per-step footprint exceeds L2"},
         "roofline": {"bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
-                     "kernel": "rrs gemm_kernel (tcgen05 kind::i8)", "peak_source": src + " (2 x bf16 burst)"},
+                     "kernel": "rrs gemm_kernel (tcgen05 kind::i8)", "peak_source": src + " (2 x bf16 burst)",
+                     "traffic_note": "DRAM bytes per GEMM launch, mean of the 3 layers (ncu)"},
         "prep": {"ms_per_layer": [round(x, 5) for x in prep_ms], "algorithmic_GBps": round(prep_gbs, 1),
                  "hbm_frac": round(prep_gbs / hbm_peak, 4)},
         "gemm": {"ms_per_layer": [round(x, 5) for x in gemm_ms], "TOPS": round(gemm_tops, 1)},
         "e2e": e2e,
+        "expanded_weights": expanded,
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
     }
