@@ -101,6 +101,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(x: float, pg, device) -> float:
+    """The largest of every rank's x (all ranks get it); x itself with no process group."""
+    if pg is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Operations of all ranks (each runs its own replica) over the slowest rank's time, in TOPS."""
+    return ops_per_step * steps * world / (ms * 1e-3) / 1e12
+
+
+def activation_sample(i: int, rank: int) -> int:
+    """Seed offset of the i-th activation set of a rank: replicas never share a batch."""
+    return 2 + i + 10 * rank
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -134,7 +153,7 @@ def run_ours(args):
         qW, sw = rrs.prepare_weights(W, perm, L.had_block)
         qW8 = rrs.expand_weights(qW)          # secondary path: weights one code per byte
         del W
-        xs = [wl.make_activations(L, sample=2 + i + 10 * rank).to(dev) for i in range(N_XSETS)]
+        xs = [wl.make_activations(L, sample=activation_sample(i, rank)).to(dev) for i in range(N_XSETS)]
         st = dict(L=L, perm=perm, qW=qW, qW8=qW8, sw=sw, xs=xs,
                   qX=torch.empty((L.M, L.K // 2), dtype=torch.uint8, device=dev),
                   s=torch.empty(L.K // L.G, dtype=torch.float32, device=dev),
@@ -189,13 +208,10 @@ def run_ours(args):
     prep_ms = [sum(evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(K)) / K for j in range(len(state))]
     gemm_ms = [sum(evs[i][j][1].elapsed_time(evs[i][j][2]) for i in range(K)) / K for j in range(len(state))]
 
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, pg, dev)
 
     ops_step = sum(st["L"].ops for st in state)
-    value = ops_step * K * world / (ms * 1e-3) / 1e12
+    value = whole_job_tops(ops_step, K, world, ms)
 
     # ---- secondary: the same step with the weights expanded offline to the int8
     # operand (rrs_expand_weights + RRS_W_EXPANDED); same codes, same results.
@@ -224,14 +240,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     # per-layer GEMM times from the last step's events (all steps are alike)
     xgemm = [xg[j][0].elapsed_time(xg[j][1]) for j in range(len(state))]
-    xms = xa.elapsed_time(xb)
-    if pg:
-        t = torch.tensor([xms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        xms = float(t.item())
+    xms = max_over_ranks(xa.elapsed_time(xb), pg, dev)
     for st in state:
         rrs.check_workspace(st["ws"])
-    expanded = {"value": round(ops_step * Kx * world / (xms * 1e-3) / 1e12, 2), "unit": UNIT, "steps": Kx,
+    expanded = {"value": round(whole_job_tops(ops_step, Kx, world, xms), 2), "unit": UNIT, "steps": Kx,
                 "gemm_ms_per_layer_last_step": [round(x, 5) for x in xgemm],
                 "weights": "INT4 codes stored one per byte as 16 q (rrs_expand_weights); 2x weight bytes"}
 
@@ -259,12 +271,8 @@ def run_ours(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        ems = a.elapsed_time(b)
-        if pg:
-            t = torch.tensor([ems], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": ops_step * Ke * world / (ems * 1e-3) / 1e12, "unit": UNIT,
+        ems = max_over_ranks(a.elapsed_time(b), pg, dev)
+        e2e = {"value": whole_job_tops(ops_step, Ke, world, ems), "unit": UNIT,
                "h2d_bytes_per_step": sum(st["L"].M * st["L"].K * 2 for st in state),
                "d2h_bytes_per_step": sum(st["L"].M * st["L"].N * 4 for st in state),
                "steps": Ke}
