@@ -380,6 +380,87 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def _time_ms(fn, iters: int = 20) -> float:
+    """Mean device time of fn() in ms (CUDA events on the current stream, 3 warm-up calls)."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def run_report(args):
+    """The other configurations: group-size sweep (cost and output error of RRS and of
+    plain Runtime Smooth against the unquantised fp32 GEMM), the 8B down projection,
+    the 70B layers and the 70B decode token counts.  One JSON line; not the bench line."""
+    import activation_smoothing_b200 as rrs
+    from activation_smoothing_b200 import workloads as wl
+
+    torch.backends.cuda.matmul.allow_tf32 = False
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    out = {"report": "RRS W4A4 linear: other configurations", "sweep": [], "layers": []}
+
+    def layer_times(L, X, W, n, flags=0, iters=20):
+        perm = rrs.calibrate_perm(wl.make_activations(L, sample=1, M=min(L.M, 512)).to(dev), n)
+        qW, sw = rrs.prepare_weights(W, perm, n, flags)
+        qX = torch.empty((L.M, L.K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty(L.K // L.G, dtype=torch.float32, device=dev)
+        st = torch.empty(L.M, dtype=torch.float32, device=dev)
+        Y = torch.empty((L.M, L.N), dtype=torch.float32, device=dev)
+        ws = rrs.make_workspace(L.M, L.N, L.K, L.G, n, flags, device=dev)
+        prep = _time_ms(lambda: rrs.smooth_quant(X, perm, L.G, n, flags, qX=qX, s=s, scale_t=st, ws=ws), iters)
+        gemm = _time_ms(lambda: rrs.w4a4_gemm(qX, s, st, qW, sw, L.G, Y=Y, ws=ws, flags=rrs.WS_HOLDS_A8), iters)
+        rrs.smooth_quant(X, perm, L.G, n, flags, qX=qX, s=s, scale_t=st, ws=ws)
+        rrs.w4a4_gemm(qX, s, st, qW, sw, L.G, Y=Y, ws=ws, flags=rrs.WS_HOLDS_A8)
+        rrs.check_workspace(ws)
+        return prep, gemm, Y
+
+    # group-size sweep on the K=4096, N=14336, M=2048 layer
+    base = wl.Layer("sweep", 2048, 4096, 14336, 128, 4096, seed=4242)
+    X = wl.make_activations(base).to(dev)
+    W = wl.make_weights(base).to(dev)
+    Yref = X.float() @ W.float().t()
+    nref = torch.linalg.vector_norm(Yref).item()
+    for G in (128, 256, 512, 4096):
+        for name, n in (("RRS", 4096), ("RS", 1)):
+            L = wl.Layer("sweep", 2048, 4096, 14336, G, n, seed=4242)
+            prep, gemm, Y = layer_times(L, X, W, n)
+            err = torch.linalg.vector_norm(Y - Yref).item() / nref
+            out["sweep"].append({"G": G, "method": name, "prep_us": round(prep * 1e3, 2), "gemm_us": round(gemm * 1e3, 2),
+                                 "TOPS": round(L.ops / ((prep + gemm) * 1e-3) / 1e12, 1),
+                                 "rel_frobenius_error_vs_fp32_gemm": float(f"{err:.5g}")})
+    del X, W, Yref
+    torch.cuda.empty_cache()
+
+    names = ["llama3_8b_down", "llama3_70b_qo", "llama3_70b_gateup", "llama3_70b_down",
+             "llama3_70b_qo_decode_m1", "llama3_70b_qo_decode_m8", "llama3_70b_qo_decode_m16",
+             "llama3_70b_gateup_decode_m1", "llama3_70b_gateup_decode_m16",
+             "llama3_70b_down_decode_m1", "llama3_70b_down_decode_m16"]
+    for nm in names:
+        if nm not in wl.LAYERS:
+            continue
+        L = wl.LAYERS[nm]
+        X = wl.make_activations(L).to(dev)
+        W = wl.make_weights(L).to(dev)
+        prep, gemm, _ = layer_times(L, X, W, L.had_block)
+        int8_peak, hbm_peak, _ = peaks()
+        wbytes = L.N * L.K // 2
+        out["layers"].append({"layer": nm, "M": L.M, "K": L.K, "N": L.N, "G": L.G, "n": L.had_block,
+                              "prep_us": round(prep * 1e3, 2), "gemm_us": round(gemm * 1e3, 2),
+                              "TOPS": round(L.ops / ((prep + gemm) * 1e-3) / 1e12, 2),
+                              "gemm_frac_int8_peak": round(L.ops / (gemm * 1e-3) / 1e12 / int8_peak, 4),
+                              "gemm_weight_GBps": round(wbytes / (gemm * 1e-3) / 1e9, 1)})
+        del X, W
+        torch.cuda.empty_cache()
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -390,10 +471,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--report", action="store_true",
+                    help="print the other configurations (group sweep, 8B down, 70B, decode) instead")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.report:
+        run_report(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
