@@ -64,8 +64,6 @@ constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
 constexpr int NTHREADS = 512;
 constexpr int UNPACK_WARPS = 2;
 constexpr int EPI_WARPS = 12;
-constexpr uint32_t kBiasBits = 0x4B400000u;   // 1.5 * 2^23
-constexpr float kBias = 12582912.0f;
 
 struct Args {
     const float* s;
@@ -129,7 +127,6 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
         mbar_arrive(&tempty[0]);
         mbar_arrive(&tempty[1]);
     }
-    const float2 negb = make_float2(-kBias, -kBias);
     const float2 sixteenth = make_float2(0.0625f, 0.0625f);
     uint32_t gc = 0;
     bool ok = true;
@@ -164,10 +161,8 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
                 for (int i = 0; i < 16; ++i) {
                     const uint32_t* rr = i < 8 ? r : r2;
                     const int ii = i & 7;
-                    // bits of 1.5 * 2^23 + 16 P as a float, minus 1.5 * 2^23: exact 16 P
-                    const float2 f = make_float2(__uint_as_float(rr[2 * ii] + kBiasBits),
-                                                 __uint_as_float(rr[2 * ii + 1] + kBiasBits));
-                    const float2 p16 = __fadd2_rn(f, negb);
+                    // |16 P| <= 2^22: the int32 -> fp32 conversion is exact
+                    const float2 p16 = make_float2(__int2float_rn((int)rr[2 * ii]), __int2float_rn((int)rr[2 * ii + 1]));
                     if (DEBUG_P) acc[8 * c + i] = __ffma2_rn(p16, sixteenth, acc[8 * c + i]);  // exact ints
                     else acc[8 * c + i] = __ffma2_rn(s2, p16, acc[8 * c + i]);
                 }

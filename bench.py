@@ -32,9 +32,9 @@ UNIT = "TOPS"
 N_XSETS = 4            # distinct activation buffers per layer, rotated between steps
 # DRAM bytes (read + write) per GEMM launch, mean over the q/o, k/v and gate/up
 # launches of one step, from the ncu capture summarised in
-# profiles/gemm_kernel_llama3_8b.md.  Must go back to None whenever gemm_kernel
-# changes until it is captured again.
-GEMM_TRAFFIC_BYTES = 44.4e6
+# profiles/gemm_kernel_llama3_8b.md.  None whenever gemm_kernel has changed since
+# that capture.
+GEMM_TRAFFIC_BYTES = None
 
 
 def peaks():
