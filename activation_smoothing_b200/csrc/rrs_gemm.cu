@@ -24,11 +24,13 @@
 //                acc += s_g * P_g (fp32, packed f32x2); per tile,
 //                Y = acc * scale_t * scale_w
 //
-// Exact int32 -> fp32 without a conversion instruction: adding the bit pattern
-// of 1.5 * 2^23 to the int32 partial 16 * P_g gives the bits of the float
-// 1.5 * 2^23 + 16 * P_g exactly (|16 P_g| <= 2^22), and one fp32 subtraction
-// recovers 16 * P_g (exact for |16 P_g| <= 2^22, i.e. groups of up to 4096 k).  Longer groups are promoted in 4096-wide
-// blocks with the same s_g.
+// Exact promotion: the weight operand holds 16 q, so a group's int32 sum is
+// 16 * P_g with |16 P_g| <= 16 * 64 * 4096 = 2^22 for groups of up to 4096 k;
+// its int32 -> fp32 conversion is then exact.  Longer groups are promoted in
+// 4096-wide blocks with the same s_g.
+//
+// A second kernel (gemm_w8_kernel, below) takes the weights already expanded
+// to that int8 operand and needs no unpack warps.
 //
 // k order: inside each 32-wide k chunk both operands store the codes in the
 // order 0,2,4,6,1,3,5,7, 8,10,... (what a nibble mask produces); the integer
