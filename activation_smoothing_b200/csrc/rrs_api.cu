@@ -149,7 +149,7 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
 
 rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
                                const float* scale_w, int M, int N, int K, int G, float* Y, int32_t* P,
-                               void* ws, unsigned flags, cudaStream_t st) {
+                               void* ws, size_t ws_bytes, unsigned flags, cudaStream_t st) {
     int8_t* qX8 = reinterpret_cast<int8_t*>(static_cast<unsigned char*>(ws) + ws_a8_offset());
     if (!(flags & RRS_WS_HOLDS_A8)) {
         cudaError_t e = rrs::launch_expand(qX, qX8, M, K, st);
@@ -169,6 +169,11 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
     gl.P = P;
     gl.err = reinterpret_cast<uint32_t*>(ws);
     gl.w_expanded = (flags & RRS_W_EXPANDED) != 0;
+    // Room after the int8 operand (the activation scratch, dead once the
+    // activation kernels have run) takes split-k partial sums for small M.
+    const size_t used = ws_bytes_gemm(M, K);
+    gl.part = ws_bytes > used ? reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + used) : nullptr;
+    gl.part_bytes = ws_bytes > used ? ws_bytes - used : 0;
     cudaError_t e = rrs::launch_gemm(gl, st);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM kernel");
     return RRS_OK;
@@ -215,11 +220,17 @@ rrs_status noalloc_scratch(void** out) {
 extern "C" {
 
 size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags) {
-    (void)N;
     (void)G;
     if (M < 1 || K < 1) return kHeaderBytes;
     const int n = (flags & RRS_NO_ROTATE) ? 1 : had_block;
-    return ws_bytes_full(M, K, n);
+    size_t b = ws_bytes_full(M, K, n);
+    if (M <= rrs::kSplitRoomMaxM && N > 0) {
+        // split-k partial sums share the space after the int8 operand with the scratch
+        const size_t room = align256((size_t)rrs::kSplitRoom * M * N * 4);
+        const size_t after = b - ws_bytes_gemm(M, K);
+        if (room > after) b += room - after;
+    }
+    return b;
 }
 
 rrs_status rrs_prepare_weights(const void* W, int N, int K, int had_block, const int32_t* perm, uint8_t* qW,
@@ -291,7 +302,7 @@ rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t
     if (r != RRS_OK) return r;
     r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
-    return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws, flags,
+    return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws, ws_bytes, flags,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -338,7 +349,7 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, in
     if (r != RRS_OK) return r;
     r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
-    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws,
+    return launch_gemm_checked(qX, nullptr, nullptr, qW, nullptr, M, N, K, G, nullptr, P, ws, ws_bytes,
                                flags & RRS_W_EXPANDED, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -76,6 +76,8 @@ struct Args {
     int32_t* P;          // debug partials [K/G, M, N] or null
     uint32_t* err;
     uint64_t limit_ns;
+    int S;               // k splits per tile (1: none); each work item is (tile, split)
+    float* part;         // S > 1: [S, M, N] fp32 partial sums (x 1/16), reduced by splitk_reduce_kernel
 };
 
 __device__ __forceinline__ uint32_t sw128_off(int row, int lc) {
@@ -116,11 +118,12 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 // sums of this warp's 32 rows x 64 columns from TMEM, promote them exactly to
 // fp32 and accumulate s_g * P_g; at the end of a tile apply scale_t * scale_w
 // and store Y (or, in debug mode, store the exact per-group partials).
-template <bool DEBUG_P>
+template <bool DEBUG_P, bool SPLIT>
 __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint64_t* tfull, uint64_t* tempty,
                                               const float* s_sm, volatile int* abortv, int warp, int lane,
-                                              int ntiles, int nmb, int NPB) {
+                                              int nwork, int nmb, int NPBS) {
     // ------------------------------------------------------------ epilogue
+    const int GS = SPLIT ? g.S : 1;               // k splits per tile
     const int quarter = warp & 3;
     const int cgrp = (warp - 4) >> 2;             // 0..2: 64-column slice of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
@@ -132,14 +135,17 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
     const float2 sixteenth = make_float2(0.0625f, 0.0625f);
     uint32_t gc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    for (int w = blockIdx.x; w < nwork && ok; w += gridDim.x) {
+        const int tile = w / GS;
+        const int sp = w % GS;
+        const int pb0 = sp * NPBS;                    // first promotion block of this k split
         const int m0 = (tile % nmb) * BM;
         const int n0 = (tile / nmb) * BN;
         float2 acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
         const int row = m0 + 32 * quarter + lane;
-        for (int pb = 0; pb < NPB; ++pb, ++gc) {
+        for (int pb = pb0; pb < pb0 + NPBS; ++pb, ++gc) {
             const int buf = gc & 1;
             if (!(ok = mbar_wait_bounded(&tfull[buf], (gc >> 1) & 1u, abortv, g.err, kErrGemmTimeout,
                                          g.limit_ns)))
@@ -190,12 +196,16 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
             const float2 swl = make_float2(cl < g.N ? g.scale_w[cl] : 0.0f, cl + 1 < g.N ? g.scale_w[cl + 1] : 0.0f);
             const float st = row < g.M ? g.scale_t[row] : 0.0f;
             const float2 st2 = make_float2(st, st);
-            float* yrow = g.Y + (size_t)row * g.N;
+            // one k split of several: its partial sum (x 1/16) goes to the workspace and
+            // splitk_reduce_kernel adds the splits in order and applies the scales
+            const bool split = SPLIT && GS > 1;
+            float* ybase = split ? g.part + (size_t)sp * g.M * g.N : g.Y;
+            float* yrow = ybase + (size_t)row * g.N;
             // Each lane owns one row, so a warp's store touches 32 rows.  Whole
             // 32-byte sectors per lane (8 columns, one 256-bit store) keep the
             // L2 from merging partial sectors; ragged edges, N % 8 != 0 and a Y
             // not 32-byte aligned fall back to scalar stores.
-            const bool v8 = (g.N & 7) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 31u) == 0;
+            const bool v8 = (g.N & 7) == 0 && (reinterpret_cast<uintptr_t>(ybase) & 31u) == 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float2 y[4];
@@ -204,7 +214,8 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
                     const int i = 4 * j + q;
                     const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i),
                                                   __shfl_sync(0xffffffffu, swl.y, i));
-                    y[q] = __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
+                    y[q] = split ? __fmul2_rn(acc[i], sixteenth)
+                                 : __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
                 }
                 const int col = n0 + col0 + 8 * j;
                 if (row < g.M) {
@@ -226,7 +237,7 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
     }
 }
 
-template <bool DEBUG_P>
+template <bool DEBUG_P, bool SPLIT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
@@ -251,6 +262,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int KB = K / BK;
     const int NPB = K / g.PB;          // promotion blocks per tile
     const int kb_per_pb = g.PB / BK;
+    const int GS = SPLIT ? g.S : 1;    // k splits per tile
+    const int KBS = KB / GS;          // k-blocks per work item (the host makes S divide NPB)
     const int nmb = (g.M + BM - 1) / BM;
     const int nnb = (g.N + BN - 1) / BN;
     const int ntiles = nmb * nnb;
@@ -291,28 +304,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // One thread, two independent streams: packed weight tiles (bounded
             // only by the unpack freeing a slot) and activation tiles (bounded by
             // the MMA freeing a stage).  Neither waits behind the other.
-            const uint32_t my_tiles = blockIdx.x < (unsigned)ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-            const uint32_t total = my_tiles * KB;
+            const int nwork = ntiles * GS;
+            const uint32_t my_items = blockIdx.x < (unsigned)nwork ? (nwork - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+            const uint32_t total = my_items * KBS;
             uint32_t itB = 0, itA = 0;
+            // position of each stream: work item, its tile and first k-block, k-block within it
+            int wB = blockIdx.x, wA = blockIdx.x;
+            int tileB = wB / GS, tileA = wA / GS;
+            int kb0B = (wB % GS) * KBS, kb0A = (wA % GS) * KBS;
+            int kkB = 0, kkA = 0;
             uint64_t t0 = 0;
             uint32_t idle = 0;
             bool ok = true;
             while (itB < total || itA < total) {
                 bool progress = false;
                 if (itB < total && mbar_test_wait(&pempty[itB % NP], ((itB / NP) & 1u) ^ 1u)) {
-                    const int tile = blockIdx.x + (itB / KB) * gridDim.x;
                     const int ps = itB % NP;
                     arrive_expect_tx(&pfull[ps], BP_BYTES);
-                    tma_load_2d(smem + OFF_BP + ps * BP_BYTES, &tmB, (itB % KB) * (BK / 2), (tile / nmb) * BN,
+                    tma_load_2d(smem + OFF_BP + ps * BP_BYTES, &tmB, (kb0B + kkB) * (BK / 2), (tileB / nmb) * BN,
                                 &pfull[ps]);
+                    if (++kkB == KBS) {
+                        kkB = 0;
+                        wB += gridDim.x;
+                        tileB = wB / GS;
+                        kb0B = (wB % GS) * KBS;
+                    }
                     ++itB;
                     progress = true;
                 }
                 if (itA < total && mbar_test_wait(&mempty[itA % NS], ((itA / NS) & 1u) ^ 1u)) {
-                    const int tile = blockIdx.x + (itA / KB) * gridDim.x;
                     const int ms = itA % NS;
                     arrive_expect_tx(&afull[ms], A_BYTES);
-                    tma_load_2d(smem + OFF_A + ms * A_BYTES, &tmA, (itA % KB) * BK, (tile % nmb) * BM, &afull[ms]);
+                    tma_load_2d(smem + OFF_A + ms * A_BYTES, &tmA, (kb0A + kkA) * BK, (tileA % nmb) * BM, &afull[ms]);
+                    if (++kkA == KBS) {
+                        kkA = 0;
+                        wA += gridDim.x;
+                        tileA = wA / GS;
+                        kb0A = (wA % GS) * KBS;
+                    }
                     ++itA;
                     progress = true;
                 }
@@ -345,8 +374,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             constexpr uint32_t idesc = idesc_i8(BM, BN);
             uint32_t it = 0, gc = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+            for (int w = blockIdx.x; w < ntiles * GS && ok; w += gridDim.x) {
+                for (int kb = 0; kb < KBS; ++kb, ++it) {
                     const bool first = (kb % kb_per_pb) == 0;
                     const bool last = (kb % kb_per_pb) == kb_per_pb - 1;
                     const int buf = gc & 1;
@@ -382,8 +411,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int r0 = p >> 2;                     // 0..15
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+            for (int w = blockIdx.x; w < ntiles * GS && ok; w += gridDim.x) {
+                for (int kb = 0; kb < KBS; ++kb, ++it) {
                     const int ps = it % NP;
                     const uint32_t pph = (it / NP) & 1u;
                     const int ms = it % NS;
@@ -420,7 +449,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
     } else {
-        epilogue_role<DEBUG_P>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
+        epilogue_role<DEBUG_P, SPLIT>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
     }
     tc_fence_before();
     __syncthreads();
@@ -450,7 +479,7 @@ static_assert(SMEM <= 227 * 1024, "shared memory budget");
 static_assert(OFF_B % 1024 == 0 && B8_BYTES % 1024 == 0, "128-byte-swizzled tiles need 1024-byte alignment");
 }  // namespace w8
 
-template <bool DEBUG_P>
+template <bool DEBUG_P, bool SPLIT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
@@ -471,6 +500,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int KB = g.K / BK;
     const int NPB = g.K / g.PB;
     const int kb_per_pb = g.PB / BK;
+    const int GS = SPLIT ? g.S : 1;
+    const int KBS = KB / GS;
     const int nmb = (g.M + BM - 1) / BM;
     const int nnb = (g.N + BN - 1) / BN;
     const int ntiles = nmb * nnb;
@@ -503,8 +534,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 0 || warp == 2 || warp == 3) {
         // -------------------------------------------------------- TMA
         const uint32_t p = warp == 0 ? 0u : (uint32_t)(warp - 1);
-        const uint32_t my_tiles = blockIdx.x < (unsigned)ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-        const uint32_t total = my_tiles * KB;
+        const int nwork = ntiles * GS;
+        const uint32_t my_items = blockIdx.x < (unsigned)nwork ? (nwork - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        const uint32_t total = my_items * KBS;
         uint32_t last = 0xFFFFFFFFu;          // last stage this warp loaded
         bool ok = true;
         for (uint32_t it = p; it < total; it += w8::NPROD) {
@@ -517,8 +549,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ok = false;
                 break;
             }
-            const int tile = blockIdx.x + (int)(it / KB) * gridDim.x;
-            const int kb = (int)(it % KB);
+            const int w = blockIdx.x + (int)(it / KBS) * gridDim.x;
+            const int tile = w / GS;
+            const int kb = (w % GS) * KBS + (int)(it % KBS);
             if (lane == 0) arrive_expect_tx(&full[st], A_BYTES + B8_BYTES);
             __syncwarp();
             if (lane < 2) {
@@ -541,8 +574,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             constexpr uint32_t idesc = idesc_i8(BM, BN);
             uint32_t it = 0, gc = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+            for (int w = blockIdx.x; w < ntiles * GS && ok; w += gridDim.x) {
+                for (int kb = 0; kb < KBS; ++kb, ++it) {
                     const bool first = (kb % kb_per_pb) == 0;
                     const bool lastk = (kb % kb_per_pb) == kb_per_pb - 1;
                     const int buf = gc & 1;
@@ -573,13 +606,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
         }
     } else {
-        epilogue_role<DEBUG_P>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
+        epilogue_role<DEBUG_P, SPLIT>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// Y = (sum over splits of the partial sums, in split order) * scale_t * scale_w.
+// The partials already carry the factor 1/16, so the products are applied in
+// the order of the unsplit epilogue.
+__global__ void splitk_reduce_kernel(const float* part, int S, int M, int N, const float* scale_t,
+                                     const float* scale_w, float* Y) {
+    const size_t total = (size_t)M * N;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        float a = part[i];
+        for (int sp = 1; sp < S; ++sp) a = __fadd_rn(a, part[(size_t)sp * total + i]);
+        const int m = (int)(i / (size_t)N);
+        const int n = (int)(i % (size_t)N);
+        Y[i] = __fmul_rn(__fmul_rn(a, scale_t[m]), scale_w[n]);
     }
 }
 
@@ -661,24 +709,41 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int ntiles = ((gl.M + BM - 1) / BM) * ((gl.N + BN - 1) / BN);
-    const int grid = ntiles < nsm ? ntiles : nsm;
+    // Few tiles (decode token counts): split k over whole promotion blocks so that
+    // every SM streams weights, if the workspace has room for the partial sums.
+    int S = 1;
+    if (gl.P == nullptr && gl.part != nullptr && gl.M <= kSplitRoomMaxM && ntiles < nsm) {
+        const int npb = gl.K / a.PB;
+        for (int c = 2; c <= kSplitRoom; ++c)
+            if (npb % c == 0 && (long)ntiles * c <= 4L * nsm && (size_t)c * gl.M * gl.N * 4 <= gl.part_bytes) S = c;
+    }
+    a.S = S;
+    a.part = S > 1 ? gl.part : nullptr;
+    const int nwork = ntiles * S;
+    const int grid = nwork < nsm ? nwork : nsm;
     cudaError_t e;
     if (gl.w_expanded) {
-        auto kern = gl.P ? gemm_w8_kernel<true> : gemm_w8_kernel<false>;
+        auto kern = gl.P ? gemm_w8_kernel<true, false> : (S > 1 ? gemm_w8_kernel<false, true> : gemm_w8_kernel<false, false>);
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w8::SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, w8::SMEM, stream>>>(tmA, tmB, a);
     } else if (gl.P) {
-        auto kern = gemm_kernel<true>;
+        auto kern = gemm_kernel<true, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
     } else {
-        auto kern = gemm_kernel<false>;
+        auto kern = S > 1 ? gemm_kernel<false, true> : gemm_kernel<false, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
     }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || S == 1) return e;
+    const size_t total = (size_t)gl.M * gl.N;
+    size_t blocks = (total + 255) / 256;
+    if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
+    splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(gl.part, S, gl.M, gl.N, gl.scale_t, gl.scale_w, gl.Y);
     return cudaGetLastError();
 }
 

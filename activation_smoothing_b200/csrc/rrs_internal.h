@@ -36,7 +36,14 @@ struct GemmLaunch {
     int32_t* P;             // [K/G, M, N] debug partials (null in normal mode)
     uint32_t* err;          // workspace error word
     bool w_expanded;        // qW holds the expanded operand written by launch_expand_weights
+    float* part;            // workspace room for split-k partial sums (may be null)
+    size_t part_bytes;
 };
+
+// Token counts up to this may split k across CTAs; the workspace then holds
+// up to kSplitRoom * M * N fp32 partial sums after the int8 operand.
+constexpr int kSplitRoomMaxM = 16;
+constexpr int kSplitRoom = 16;
 
 // Fast activation path (K % 2048 == 0): rotation + reorder + group max into an
 // fp32 scratch, then smoothing + quantisation.

@@ -144,6 +144,32 @@ def test_y_not_32_byte_aligned_matches(rrs, M, N):
     assert torch.all(big[:4] == 0) and torch.all(big[4 + M * N:] == 0)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 8192, 8192), (16, 2048, 28672), (8, 1000, 4096)])
+def test_split_k_for_small_m(rrs, M, N, K):
+    """Token counts up to 16 split k across CTAs when the workspace has room: Y within the
+    tolerance of the oracle and of the unsplit kernel (a workspace sized without room)."""
+    G = 128
+    rng = np.random.default_rng(M * 7 + K)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = (rng.random(K // G, dtype=np.float32) + 0.5).astype(np.float32)
+    st = rng.random(M, dtype=np.float32)
+    sw = rng.random(N, dtype=np.float32)
+    args = [torch.from_numpy(a).to(DEV) for a in (qX, s, st, qW, sw)]
+    big = rrs.workspace_size(M, N, K, G, 1)
+    small = rrs.workspace_size(M, 0, K, G, 1)
+    assert big > small
+    Y_split = rrs.w4a4_gemm(*args, G, ws=rrs.make_workspace(M, N, K, G, 1))
+    Y_one = rrs.w4a4_gemm(*args, G, ws=rrs.make_workspace(M, 0, K, G, 1))
+    torch.cuda.synchronize()
+    Yo, B = oracle.linear_rows(qX, s, st, qW, sw, G)
+    for Y in (Y_split, Y_one):
+        ok = oracle.y_tolerance_ok(Y.cpu().numpy(), Yo, B)
+        assert ok.all(), f"{np.count_nonzero(~ok)} outside tolerance"
+    d = (Y_split - Y_one).abs().max().item()
+    assert d <= 1e-5 * Y_one.abs().max().item()
+
+
 def test_partials_extreme_codes(rrs):
     """All codes -8 or 7 (|P_g| at its maximum 64 G) stay exact."""
     rng = np.random.default_rng(1)
