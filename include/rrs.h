@@ -97,7 +97,11 @@ typedef enum {
  * first use), then the int8 copy of the activation codes that the GEMM's
  * tensor cores read (M*K bytes), then, when K is a multiple of 2048, the
  * reordered fp32 activations X' that pass between the two activation kernels
- * (M*K*4 bytes).  rrs_w4a4_gemm alone needs only the first two parts. */
+ * (M*K*4 bytes).  For M <= 16 the space after the int8 operand is at least
+ * 16*M*N*4 bytes: the GEMM then splits k across CTAs and keeps the partial sums
+ * there (the X' scratch is dead by then).  rrs_w4a4_gemm alone needs only the
+ * first two parts; given less room it simply does not split.  One workspace
+ * must not be used by two calls in flight at the same time. */
 size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags);
 
 /* Offline weight path (summary page "Approach"; rebuttal page "Description of
