@@ -120,6 +120,14 @@ def activation_sample(i: int, rank: int) -> int:
     return 2 + i + 10 * rank
 
 
+def bench_config(names, layers, world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": "+".join(names),
+            "shapes": [dict(M=L.M, K=L.K, N=L.N, G=L.G, had=L.had_block) for L in layers],
+            "parallelism": f"replicas{world}",
+            "l2": f"activations rotate over {N_XSETS} sets per layer; per-step footprint exceeds L2"}
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -290,11 +298,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8 MMA / fp32 prep",
         "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights); weights packed INT4",
-        "config": {"workload": "+".join(names),
-                   "shapes": [dict(M=st["L"].M, K=st["L"].K, N=st["L"].N, G=st["L"].G, had=st["L"].had_block)
-                              for st in state],
-                   "parallelism": f"replicas{world}",
-                   "l2": f"activations rotate over {N_XSETS} sets per layer; per-step footprint exceeds L2"},
+        "config": bench_config(names, layers, world),
         "roofline": {"bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
                      "kernel": "rrs gemm_kernel (tcgen05 kind::i8)", "peak_source": src + " (2 x bf16 burst)",
@@ -372,7 +376,7 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_s * 1e3 / args.steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32/int (CPU oracle)",
-           "data": "synthetic", "config": {"workload": "+".join(names), "parallelism": "host"},
+           "data": "synthetic", "config": bench_config(names, layers, world),
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                             "sample": f"per step: 1 token row of each layer, prep + GEMM against {cols} "
                                       f"output columns; weights prepared untimed"},
