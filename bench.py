@@ -385,17 +385,37 @@ def run_reference(args):
 
 
 def _time_ms(fn, iters: int = 20) -> float:
-    """Mean device time of fn() in ms (CUDA events on the current stream, 3 warm-up calls)."""
-    for _ in range(3):
-        fn()
+    """Mean device time of fn() in ms.  The calls are captured in a CUDA graph and the
+    graph is replayed (CUDA events on the current stream), so that host launch overhead
+    does not hide the kernel time of small (decode) calls; eager calls if capture fails."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
-        fn()
-    b.record()
-    torch.cuda.synchronize()
-    return a.elapsed_time(b) / iters
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(iters):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+    except Exception:
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
 
 
 def run_report(args):

@@ -170,6 +170,49 @@ def test_split_k_for_small_m(rrs, M, N, K):
     assert d <= 1e-5 * Y_one.abs().max().item()
 
 
+@pytest.mark.parametrize("M,N,K,G", [(4, 3000, 8192, 512), (16, 1536, 4096, 1024), (2, 704, 16384, 8192)])
+def test_split_k_group_sizes_and_expanded_weights(rrs, M, N, K, G):
+    """Split k with groups wider than one k-block (and G > 4096, promoted in 4096-wide
+    pieces), for packed and expanded weights: both within the oracle's tolerance and
+    bit-identical to each other (same kernels, same split)."""
+    rng = np.random.default_rng(M + N + G)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = (rng.random(K // G, dtype=np.float32) + 0.5).astype(np.float32)
+    st = rng.random(M, dtype=np.float32)
+    sw = rng.random(N, dtype=np.float32)
+    qXd, sd, std, qWd, swd = (torch.from_numpy(a).to(DEV) for a in (qX, s, st, qW, sw))
+    ws = rrs.make_workspace(M, N, K, G, 1)
+    Y = rrs.w4a4_gemm(qXd, sd, std, qWd, swd, G, ws=ws)
+    Y8 = rrs.w4a4_gemm(qXd, sd, std, rrs.expand_weights(qWd), swd, G, ws=ws, flags=rrs.W_EXPANDED)
+    torch.cuda.synchronize()
+    assert_bits_equal(Y8, Y, "Y (expanded, split) vs Y (packed, split)")
+    Yo, B = oracle.linear_rows(qX, s, st, qW, sw, G)
+    ok = oracle.y_tolerance_ok(Y.cpu().numpy(), Yo, B)
+    assert ok.all(), f"{np.count_nonzero(~ok)} outside tolerance"
+
+
+@pytest.mark.parametrize("M,K,G,n,flags", [(1, 2048, 128, 2048, 0), (3, 4096, 256, 4096, 0), (16, 8192, 128, 8192, 0),
+                                            (5, 14336, 128, 2048, 0), (2, 4096, 128, 4096, 1), (4, 2048, 512, 1024, 2),
+                                            (16, 2048, 2048, 2048, 0)])
+def test_activation_path_small_m_repeated_calls(rrs, M, K, G, n, flags):
+    """Decode-sized token counts on the fast activation path: codes, s and scale_t
+    bit-exact with the oracle, over repeated calls on one workspace with different M."""
+    L = wl.Layer("small", M, K, 256, G, n, seed=M * 31 + K)
+    unit = bool(flags & rrs.FORCE_UNIT_SCALES)
+    n_eff = 1 if flags & rrs.NO_ROTATE else n
+    perm = wl.random_perm(K, M)
+    ws = rrs.make_workspace(16, 256, K, G, n, flags)
+    for rep, m in enumerate((M, max(1, M // 2), M)):
+        X = wl.make_activations(L, sample=rep, M=m)
+        qX, s, st = rrs.smooth_quant(X.to(DEV), perm.to(DEV), G, n, flags, ws=ws)
+        rrs.check_workspace(ws)
+        _, oqX, os_, ost = oracle.smooth_quant(X, G, n_eff, perm.numpy(), unit_scales=unit)
+        assert_bits_equal(s, os_, f"s (call {rep}, M={m})")
+        assert_bits_equal(st, ost, f"scale_t (call {rep}, M={m})")
+        assert_bits_equal(qX, oqX, f"qX (call {rep}, M={m})")
+
+
 def test_partials_extreme_codes(rrs):
     """All codes -8 or 7 (|P_g| at its maximum 64 G) stay exact."""
     rng = np.random.default_rng(1)
