@@ -21,6 +21,7 @@ NO_ROTATE = 1
 FORCE_UNIT_SCALES = 2
 WS_HOLDS_A8 = 4
 W_EXPANDED = 8
+Y_BF16 = 16
 
 _STATUS = {
     0: "RRS_OK",
@@ -149,6 +150,17 @@ def smooth_quant(X: torch.Tensor, perm: torch.Tensor, G: int, had_block: int, fl
     return qX, s, scale_t
 
 
+def _y_flags(Y: Optional[torch.Tensor], flags: int) -> int:
+    """A bf16 Y selects the bf16 output (RRS_Y_BF16)."""
+    if Y is not None and Y.dtype == torch.bfloat16:
+        return flags | Y_BF16
+    return flags
+
+
+def _y_dtype(flags: int) -> torch.dtype:
+    return torch.bfloat16 if flags & Y_BF16 else torch.float32
+
+
 def _need_weights(qW: torch.Tensor, N: int, K: int, flags: int):
     if flags & W_EXPANDED:
         _need(qW, "qW", torch.int8, (N, K))
@@ -170,8 +182,9 @@ def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torc
     _need(s, "s", torch.float32, (K // G,))
     _need(scale_t, "scale_t", torch.float32, (M,))
     _need(scale_w, "scale_w", torch.float32, (N,))
-    Y = torch.empty((M, N), dtype=torch.float32, device=qX.device) if Y is None else Y
-    _need(Y, "Y", torch.float32, (M, N))
+    flags = _y_flags(Y, flags)
+    Y = torch.empty((M, N), dtype=_y_dtype(flags), device=qX.device) if Y is None else Y
+    _need(Y, "Y", _y_dtype(flags), (M, N))
     ws = make_workspace(M, N, K, G, 1, 0, qX.device) if ws is None else ws
     _check(lib().rrs_w4a4_gemm(_ptr(qX), _ptr(s), _ptr(scale_t), _ptr(qW), _ptr(scale_w), M, N, K, G, _ptr(Y),
                                _ptr(ws), ws.numel(), flags, _stream(stream)))
@@ -194,8 +207,9 @@ def linear(X: torch.Tensor, qW: torch.Tensor, scale_w: torch.Tensor, perm: torch
     qX = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if qX is None else qX
     s = torch.empty(max(K // G, 1), dtype=torch.float32, device=dev) if s is None else s
     scale_t = torch.empty(M, dtype=torch.float32, device=dev) if scale_t is None else scale_t
-    Y = torch.empty((M, N), dtype=torch.float32, device=dev) if Y is None else Y
-    _need(Y, "Y", torch.float32, (M, N))
+    flags = _y_flags(Y, flags)
+    Y = torch.empty((M, N), dtype=_y_dtype(flags), device=dev) if Y is None else Y
+    _need(Y, "Y", _y_dtype(flags), (M, N))
     ws = make_workspace(M, N, K, G, had_block, flags, dev) if ws is None else ws
     _check(lib().rrs_linear(_ptr(X), _ptr(qW), _ptr(scale_w), _ptr(perm), M, N, K, G, had_block, _ptr(qX),
                             _ptr(s), _ptr(scale_t), _ptr(Y), _ptr(ws), ws.numel(), flags, _stream(stream)))
@@ -211,12 +225,13 @@ def linear_from_host(X_host: torch.Tensor, X_dev: torch.Tensor, qW: torch.Tensor
     N = qW.shape[0]
     if X_host.device.type != "cpu" or Y_host.device.type != "cpu":
         raise ValueError("X_host and Y_host must be host tensors")
-    if X_host.dtype != torch.float16 or Y_host.dtype != torch.float32:
-        raise TypeError("X_host must be fp16 and Y_host fp32")
+    flags = _y_flags(Y_dev, flags)
+    if X_host.dtype != torch.float16 or Y_host.dtype != _y_dtype(flags):
+        raise TypeError("X_host must be fp16 and Y_host of Y_dev's type (fp32 or bf16)")
     if tuple(Y_host.shape) != (M, N) or not X_host.is_contiguous() or not Y_host.is_contiguous():
         raise ValueError("host buffers must be contiguous with shapes [M, K] and [M, N]")
     _need(X_dev, "X_dev", torch.float16, (M, K))
-    _need(Y_dev, "Y_dev", torch.float32, (M, N))
+    _need(Y_dev, "Y_dev", _y_dtype(flags), (M, N))
     _check(lib().rrs_linear_from_host(_ptr(X_host), _ptr(X_dev), _ptr(qW), _ptr(scale_w), _ptr(perm), M, N, K,
                                       G, had_block, _ptr(qX), _ptr(s), _ptr(scale_t), _ptr(Y_dev), _ptr(Y_host),
                                       _ptr(ws), ws.numel(), flags, _stream(stream)))

@@ -169,6 +169,7 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
     gl.P = P;
     gl.err = reinterpret_cast<uint32_t*>(ws);
     gl.w_expanded = (flags & RRS_W_EXPANDED) != 0;
+    gl.y_bf16 = P == nullptr && (flags & RRS_Y_BF16) != 0;
     // Room after the int8 operand (the activation scratch, dead once the
     // activation kernels have run) takes split-k partial sums for small M.
     const size_t used = ws_bytes_gemm(M, K);
@@ -312,7 +313,7 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
     return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes,
-                         RRS_WS_HOLDS_A8 | (flags & RRS_W_EXPANDED), stream);
+                         RRS_WS_HOLDS_A8 | (flags & (RRS_W_EXPANDED | RRS_Y_BF16)), stream);
 }
 
 rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* qW, const float* scale_w,
@@ -329,7 +330,7 @@ rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* 
     rrs_status r = rrs_linear(X_dev, qW, scale_w, perm, M, N, K, G, had_block, qX, s, scale_t, Y_dev, ws,
                               ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
-    e = cudaMemcpyAsync(Y_host, Y_dev, (size_t)M * N * 4, cudaMemcpyDeviceToHost, st);
+    e = cudaMemcpyAsync(Y_host, Y_dev, (size_t)M * N * ((flags & RRS_Y_BF16) ? 2 : 4), cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy of Y");
     e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

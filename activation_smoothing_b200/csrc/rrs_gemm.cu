@@ -36,6 +36,7 @@
 // order 0,2,4,6,1,3,5,7, 8,10,... (what a nibble mask produces); the integer
 // sum over the chunk does not depend on the order.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -78,6 +79,7 @@ struct Args {
     uint64_t limit_ns;
     int S;               // k splits per tile (1: none); each work item is (tile, split)
     float* part;         // S > 1: [S, M, N] fp32 partial sums (x 1/16), reduced by splitk_reduce_kernel
+    bool ybf16;          // Y is bf16 [M, N] (the fp32 result rounded to nearest even)
 };
 
 __device__ __forceinline__ uint32_t sw128_off(int row, int lc) {
@@ -209,7 +211,25 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
                                  : __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
                 }
                 const int col = n0 + col0 + 8 * j;
-                if (row < g.M) {
+                if (row < g.M && g.ybf16 && !split) {
+                    // bf16 output: 8 columns = one 16-byte store
+                    __nv_bfloat16* brow = reinterpret_cast<__nv_bfloat16*>(g.Y) + (size_t)row * g.N;
+                    if ((g.N & 7) == 0 && col + 7 < g.N) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const __nv_bfloat162 b = __float22bfloat162_rn(y[q]);
+                            u[q] = *reinterpret_cast<const uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(brow + col) = make_uint4(u[0], u[1], u[2], u[3]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (col + 2 * q < g.N) brow[col + 2 * q] = __float2bfloat16_rn(y[q].x);
+                            if (col + 2 * q + 1 < g.N) brow[col + 2 * q + 1] = __float2bfloat16_rn(y[q].y);
+                        }
+                    }
+                } else if (row < g.M) {
                     if (v8 && col + 7 < g.N) {
                         asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
                                      ::"l"(yrow + col), "f"(y[0].x), "f"(y[0].y), "f"(y[1].x), "f"(y[1].y),
@@ -611,14 +631,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // The partials already carry the factor 1/16, so the products are applied in
 // the order of the unsplit epilogue.
 __global__ void splitk_reduce_kernel(const float* part, int S, int M, int N, const float* scale_t,
-                                     const float* scale_w, float* Y) {
+                                     const float* scale_w, float* Y, bool ybf16) {
     const size_t total = (size_t)M * N;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
         float a = part[i];
         for (int sp = 1; sp < S; ++sp) a = __fadd_rn(a, part[(size_t)sp * total + i]);
         const int m = (int)(i / (size_t)N);
         const int n = (int)(i % (size_t)N);
-        Y[i] = __fmul_rn(__fmul_rn(a, scale_t[m]), scale_w[n]);
+        const float y = __fmul_rn(__fmul_rn(a, scale_t[m]), scale_w[n]);
+        if (ybf16) reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(y);
+        else Y[i] = y;
     }
 }
 
@@ -710,6 +732,7 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     }
     a.S = S;
     a.part = S > 1 ? gl.part : nullptr;
+    a.ybf16 = gl.y_bf16;
     const int nwork = ntiles * S;
     const int grid = nwork < nsm ? nwork : nsm;
     cudaError_t e;
@@ -734,7 +757,8 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     const size_t total = (size_t)gl.M * gl.N;
     size_t blocks = (total + 255) / 256;
     if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
-    splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(gl.part, S, gl.M, gl.N, gl.scale_t, gl.scale_w, gl.Y);
+    splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(gl.part, S, gl.M, gl.N, gl.scale_t, gl.scale_w, gl.Y,
+                                                               gl.y_bf16);
     return cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ struct GemmLaunch {
     bool w_expanded;        // qW holds the expanded operand written by launch_expand_weights
     float* part;            // workspace room for split-k partial sums (may be null)
     size_t part_bytes;
+    bool y_bf16;            // Y is bf16 [M, N] instead of fp32
 };
 
 // Token counts up to this may split k across CTAs; the workspace then holds

@@ -91,6 +91,10 @@ typedef enum {
 #define RRS_W_EXPANDED 8u        /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host and the debug
                                     partials: qW points at the int8 operand that rrs_expand_weights
                                     wrote ([N, K] bytes) instead of the packed INT4 codes */
+#define RRS_Y_BF16 16u           /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host: Y (and Y_host)
+                                    hold bf16 [M, N] -- the fp32 result rounded to nearest even --
+                                    instead of fp32; pass the buffer cast to float *.  The pages fix
+                                    no output type; bf16 is the usual deployment type of Y. */
 
 /* Bytes of workspace the calls below need for this problem.  Layout: a
  * 256-byte header holding the kernels' error word (zero-fill it once before

@@ -213,6 +213,24 @@ def test_activation_path_small_m_repeated_calls(rrs, M, K, G, n, flags):
         assert_bits_equal(qX, oqX, f"qX (call {rep}, M={m})")
 
 
+@pytest.mark.parametrize("M,N,K", [(2048, 4096, 4096), (130, 520, 1024), (8, 2048, 8192), (33, 200, 512), (17, 203, 1024)])
+def test_bf16_output_is_rounded_fp32(rrs, M, N, K):
+    """RRS_Y_BF16: Y in bf16 equals the fp32 Y rounded to nearest even, bit for bit, on the
+    prefill kernel, the split-k path (M <= 16), ragged N and through rrs_linear."""
+    G = 128
+    L = wl.Layer("bf16", M, K, N, G, K if K <= 8192 else 2048, seed=M + N)
+    X, W = wl.make_activations(L).to(DEV), wl.make_weights(L).to(DEV)
+    perm = wl.random_perm(K, 3).to(DEV)
+    qW, sw = rrs.prepare_weights(W, perm, L.had_block)
+    ws = rrs.make_workspace(M, N, K, G, L.had_block)
+    Y32 = rrs.linear(X, qW, sw, perm, G, L.had_block, ws=ws)
+    Y16 = rrs.linear(X, qW, sw, perm, G, L.had_block, ws=ws,
+                     Y=torch.empty((M, N), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert Y16.dtype == torch.bfloat16
+    assert_bits_equal(Y16.view(torch.int16), Y32.to(torch.bfloat16).view(torch.int16), "bf16 Y")
+
+
 def test_partials_extreme_codes(rrs):
     """All codes -8 or 7 (|P_g| at its maximum 64 G) stay exact."""
     rng = np.random.default_rng(1)
