@@ -111,7 +111,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 // sums of this warp's 32 rows x 64 columns from TMEM, promote them exactly to
 // fp32 and accumulate s_g * P_g; at the end of a tile apply scale_t * scale_w
 // and store Y (or, in debug mode, store the exact per-group partials).
-template <bool DEBUG_P, bool SPLIT>
+template <bool DEBUG_P, bool SPLIT, bool YBF16>
 __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint64_t* tfull, uint64_t* tempty,
                                               const float* s_sm, volatile int* abortv, int warp, int lane,
                                               int nwork, int nmb, int NPBS) {
@@ -211,7 +211,7 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
                                  : __fmul2_rn(__fmul2_rn(__fmul2_rn(acc[i], sixteenth), st2), sw);
                 }
                 const int col = n0 + col0 + 8 * j;
-                if (row < g.M && g.ybf16 && !split) {
+                if (YBF16 && row < g.M && !split) {
                     // bf16 output: 8 columns = one 16-byte store
                     __nv_bfloat16* brow = reinterpret_cast<__nv_bfloat16*>(g.Y) + (size_t)row * g.N;
                     if ((g.N & 7) == 0 && col + 7 < g.N) {
@@ -248,7 +248,7 @@ __device__ __forceinline__ void epilogue_role(const Args& g, uint32_t tmem, uint
     }
 }
 
-template <bool DEBUG_P, bool SPLIT>
+template <bool DEBUG_P, bool SPLIT, bool YBF16>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
     } else {
-        epilogue_role<DEBUG_P, SPLIT>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
+        epilogue_role<DEBUG_P, SPLIT, YBF16>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
     }
     tc_fence_before();
     __syncthreads();
@@ -490,7 +490,7 @@ static_assert(SMEM <= 227 * 1024, "shared memory budget");
 static_assert(OFF_B % 1024 == 0 && B8_BYTES % 1024 == 0, "128-byte-swizzled tiles need 1024-byte alignment");
 }  // namespace w8
 
-template <bool DEBUG_P, bool SPLIT>
+template <bool DEBUG_P, bool SPLIT, bool YBF16>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
@@ -617,7 +617,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
         }
     } else {
-        epilogue_role<DEBUG_P, SPLIT>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
+        epilogue_role<DEBUG_P, SPLIT, YBF16>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
     }
     tc_fence_before();
     __syncthreads();
@@ -737,17 +737,23 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     const int grid = nwork < nsm ? nwork : nsm;
     cudaError_t e;
     if (gl.w_expanded) {
-        auto kern = gl.P ? gemm_w8_kernel<true, false> : (S > 1 ? gemm_w8_kernel<false, true> : gemm_w8_kernel<false, false>);
+        // (with split k the bf16 rounding happens in splitk_reduce_kernel)
+        auto kern = gl.P     ? gemm_w8_kernel<true, false, false>
+                    : S > 1  ? gemm_w8_kernel<false, true, false>
+                    : a.ybf16 ? gemm_w8_kernel<false, false, true>
+                              : gemm_w8_kernel<false, false, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w8::SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, w8::SMEM, stream>>>(tmA, tmB, a);
     } else if (gl.P) {
-        auto kern = gemm_kernel<true, false>;
+        auto kern = gemm_kernel<true, false, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
     } else {
-        auto kern = S > 1 ? gemm_kernel<false, true> : gemm_kernel<false, false>;
+        auto kern = S > 1    ? gemm_kernel<false, true, false>
+                    : a.ybf16 ? gemm_kernel<false, false, true>
+                              : gemm_kernel<false, false, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
         kern<<<grid, NTHREADS, SMEM, stream>>>(tmA, tmB, a);
