@@ -34,7 +34,7 @@ N_XSETS = 4            # distinct activation buffers per layer, rotated between 
 # launches of one step, from the ncu capture summarised in
 # profiles/gemm_kernel_llama3_8b.md.  None whenever gemm_kernel has changed since
 # that capture.
-GEMM_TRAFFIC_BYTES = None
+GEMM_TRAFFIC_BYTES = 45.8e6
 
 
 def peaks():
