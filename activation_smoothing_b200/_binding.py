@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         "rrs_linear_from_host": ([P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, Z, U, P], I),
         "rrs_w4a4_gemm_debug_partials": ([P, P, I, I, I, I, P, P, Z, U, P], I),
         "rrs_expand_weights": ([P, I, I, P, P], I),
+        "rrs_silu_mul": ([P, I, I, P, P], I),
         "rrs_channel_absmax": ([P, I, I, I, P, U, P], I),
         "rrs_perm_from_channel_max": ([P, I, P], I),
         "rrs_check_workspace": ([P, P], I),
@@ -252,6 +253,19 @@ def w4a4_gemm_debug_partials(qX: torch.Tensor, qW: torch.Tensor, G: int, P: Opti
     _check(lib().rrs_w4a4_gemm_debug_partials(_ptr(qX), _ptr(qW), M, N, K, G, _ptr(P), _ptr(ws), ws.numel(),
                                               flags & W_EXPANDED, _stream(stream)))
     return P
+
+
+def silu_mul(GU: torch.Tensor, H: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fp16 H [M, F] = silu(GU[:, :F]) * GU[:, F:] from the fused gate/up output GU fp32 [M, 2F]."""
+    M, F2 = GU.shape
+    if F2 % 2:
+        raise ValueError("GU must have an even number of columns [gate | up]")
+    F = F2 // 2
+    _need(GU, "GU", torch.float32, (M, F2))
+    H = torch.empty((M, F), dtype=torch.float16, device=GU.device) if H is None else H
+    _need(H, "H", torch.float16, (M, F))
+    _check(lib().rrs_silu_mul(_ptr(GU), M, F, _ptr(H), _stream(stream)))
+    return H
 
 
 def expand_weights(qW: torch.Tensor, qW8: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -354,6 +354,15 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, in
                                flags & RRS_W_EXPANDED, reinterpret_cast<cudaStream_t>(stream));
 }
 
+rrs_status rrs_silu_mul(const float* GU, int M, int F, void* H, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(GU);
+    RRS_REQUIRE_PTR(H);
+    if (M < 1 || F < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, F = %d", M, F);
+    cudaError_t e = rrs::launch_silu_mul(GU, M, F, H, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "silu_mul kernel");
+    return RRS_OK;
+}
+
 rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, int8_t* qW8, rrs_stream_t stream) {
     RRS_REQUIRE_PTR(qW);
     RRS_REQUIRE_PTR(qW8);

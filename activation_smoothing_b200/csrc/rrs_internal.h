@@ -70,6 +70,8 @@ cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStre
 cudaError_t launch_expand_weights(const uint8_t* qW, int8_t* qW8, int N, int K, cudaStream_t stream);
 
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream);
+// H fp16 [M, F] = silu(GU[:, :F]) * GU[:, F:], GU fp32 [M, 2F].
+cudaError_t launch_silu_mul(const float* GU, int M, int F, void* H, cudaStream_t stream);
 cudaError_t launch_divide_check(const float* a, const float* b, int n, float* q_fast, float* q_ieee,
                                 cudaStream_t stream);
 

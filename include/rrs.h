@@ -168,6 +168,16 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t *qX, const uint8_t *qW, in
  * Asynchronous on `stream`. */
 rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, int8_t *qW8, rrs_stream_t stream);
 
+/* Gated-MLP step between two RRS linears (summary page "Key results": the method is
+ * applied to every linear layer of the model, so the down projection's input is the
+ * gated activation): H[m][f] = silu(GU[m][f]) * GU[m][F + f], silu(g) = g / (1 +
+ * exp(-g)) in fp32, rounded to fp16 and saturated to +-65504.  GU fp32 [M, 2F], the
+ * output of the fused gate/up projection whose weight rows are [W_gate; W_up]; H fp16
+ * [M, F], the down projection's X.  Both device, caller-owned, 16-byte aligned.  The
+ * pages fix no activation function; SiLU is that of the LLaMA models they evaluate.
+ * Asynchronous on `stream`. */
+rrs_status rrs_silu_mul(const float *GU, int M, int F, void *H, rrs_stream_t stream);
+
 /* Calibration statistic for the reorder index: cmax[k] = max_t |X_rot[t][k]|
  * (rotation only, no reorder).  cmax fp32 [K]. */
 rrs_status rrs_channel_absmax(const void *X, int M, int K, int had_block, float *cmax,

@@ -1,0 +1,126 @@
+"""Gated MLP block on the CUDA path (needs a B200): gate/up RRS linear, SiLU * up,
+down RRS linear with a block-diagonal Hadamard.
+
+Parity is checked stage by stage.  Each linear matches the oracle as in the layer
+tests (codes bit-exact, Y within tolerance), the down projection being fed the GPU's
+own H.  SiLU * up is within one fp16 ulp of an fp64 reference: both sides round, and
+the GPU's exp is CUDA's, not the host's, so bit equality is not expected there.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_smoothing_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda")
+
+
+@pytest.fixture(scope="module")
+def rrs():
+    import activation_smoothing_b200 as m
+    m.lib()
+    return m
+
+
+def _silu_mul_ref(GU: np.ndarray) -> np.ndarray:
+    F = GU.shape[1] // 2
+    g = GU[:, :F].astype(np.float64)
+    u = GU[:, F:].astype(np.float64)
+    h = g / (1.0 + np.exp(-g)) * u
+    return np.clip(h, -65504.0, 65504.0)
+
+
+def _ulp16(x: np.ndarray) -> np.ndarray:
+    """Spacing of fp16 values at |x| (subnormal spacing below the normal range)."""
+    a = np.abs(x).astype(np.float64)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
+@pytest.mark.parametrize("M,F", [(37, 1000), (256, 14336), (5, 3)])
+def test_silu_mul_within_one_fp16_ulp(rrs, M, F):
+    g = torch.Generator().manual_seed(M + F)
+    GU = torch.randn(M, 2 * F, generator=g) * 4.0
+    GU[0, 0] = 0.0
+    GU[-1, -1] = 1e6                        # product beyond fp16: saturates
+    GU[-1, F - 1] = 1e6
+    H = rrs.silu_mul(GU.to(DEV))
+    torch.cuda.synchronize()
+    ref = _silu_mul_ref(GU.numpy())
+    got = H.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert got[-1, -1] == 65504.0
+    assert got[0, 0] == 0.0
+    err = np.abs(got - ref)
+    assert np.all(err <= _ulp16(ref) + 1e-12), float((err / _ulp16(ref)).max())
+
+
+def _linear_checked(rrs, X_dev, W, perm, G, n, rows=None):
+    """GPU RRS linear of X_dev (fp16, device) against the oracle run on the same X."""
+    M, K = X_dev.shape
+    Wd, pd = W.to(DEV), perm.to(DEV)
+    qW, sw = rrs.prepare_weights(Wd, pd, n)
+    qX, s, st = rrs.smooth_quant(X_dev, pd, G, n)
+    ws = rrs.make_workspace(M, W.shape[0], K, G, n)
+    Y = rrs.w4a4_gemm(qX, s, st, qW, sw, G, ws=ws)
+    rrs.check_workspace(ws)
+    torch.cuda.synchronize()
+    X = X_dev.cpu()
+    _, oqX, os_, ost = oracle.smooth_quant(X, G, n, perm.numpy())
+    for got, want, what in ((qX, oqX, "qX"), (s, os_, "s"), (st, ost, "scale_t")):
+        g = got.cpu().numpy()
+        assert np.array_equal(g.view(np.uint8), np.asarray(want).view(np.uint8)), what
+    _, oqW, osw = oracle.prepare_weights(W, n, perm.numpy())
+    assert np.array_equal(qW.cpu().numpy(), oqW)
+    Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
+    Yg = Y.cpu().numpy() if rows is None else Y.cpu().numpy()[rows]
+    ok = oracle.y_tolerance_ok(Yg, Yo, B)
+    assert ok.all(), f"{np.count_nonzero(~ok)} of {ok.size} outside tolerance"
+    return Y
+
+
+def test_mlp_block_stagewise_parity(rrs):
+    M, K, F, G = 64, 512, 1024, 128
+    up = wl.Layer("mlp_gu", M, K, 2 * F, G, K, seed=77)
+    down = wl.Layer("mlp_down", M, F, K, G, 512, seed=78)   # 2 Hadamard blocks of 512
+    X = wl.make_activations(up)
+    Wgu = wl.make_weights(up)
+    Wd = wl.make_weights(down)
+    perm_gu = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(up, sample=1), K))
+    GU = _linear_checked(rrs, X.to(DEV), Wgu, perm_gu, G, K)
+    H = rrs.silu_mul(GU)
+    torch.cuda.synchronize()
+    ref = _silu_mul_ref(GU.cpu().numpy())
+    assert np.all(np.abs(H.float().cpu().numpy() - ref) <= _ulp16(ref) + 1e-12)
+    perm_d = torch.from_numpy(oracle.calibrate_perm(H.cpu(), down.had_block))
+    _linear_checked(rrs, H, Wd, perm_d, G, down.had_block)
+
+
+def test_mlp_block_quality_bounded(rrs):
+    """Block output of RRS and of plain Runtime Smooth against the unquantised fp32 block
+    on the same fp16 inputs: both finite and bounded.  (The pages' RRS-over-RS ordering is
+    about real LLM activations; on this synthetic block the two are close, RS slightly
+    ahead, so the ordering is reported, not asserted.)"""
+    M, K, F, G = 256, 1024, 2048, 128
+    up = wl.Layer("mlp_gu", M, K, 2 * F, G, K, seed=91)
+    Xd = wl.make_activations(up).to(DEV)
+    Wgu = wl.make_weights(up).to(DEV)
+    Wd = wl.make_weights(wl.Layer("mlp_down", M, F, K, G, F, seed=92)).to(DEV)
+    ref = Xd.float() @ Wgu.float().t()
+    ref = (torch.nn.functional.silu(ref[:, :F]) * ref[:, F:]).half().float() @ Wd.float().t()
+    errs = {}
+    for name, n_up, n_down in (("RRS", K, F), ("RS", 1, 1)):
+        pg = rrs.calibrate_perm(wl.make_activations(up, sample=1).to(DEV), n_up)
+        qW, sw = rrs.prepare_weights(Wgu, pg, n_up)
+        GU = rrs.linear(Xd, qW, sw, pg, G, n_up)
+        H = rrs.silu_mul(GU)
+        pd = rrs.calibrate_perm(H, n_down)
+        qWd, swd = rrs.prepare_weights(Wd, pd, n_down)
+        Y = rrs.linear(H, qWd, swd, pd, G, n_down)
+        torch.cuda.synchronize()
+        errs[name] = (torch.linalg.vector_norm(Y - ref) / torch.linalg.vector_norm(ref)).item()
+    print("mlp block relative error vs fp32:", errs)
+    assert all(np.isfinite(v) and v < 0.5 for v in errs.values()), errs
