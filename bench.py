@@ -462,6 +462,34 @@ def run_report(args):
     del X, W, Yref
     torch.cuda.empty_cache()
 
+    # gated MLP block at LLaMA-3-8B sizes: gate/up linear (N = 2 x 14336), SiLU * up, down linear
+    Lgu = wl.Layer("llama3_8b_mlp_gateup", 2048, 4096, 2 * 14336, 128, 4096, seed=501)
+    Ld = wl.Layer("llama3_8b_mlp_down", 2048, 14336, 4096, 128, 2048, seed=502)
+    Xgu = wl.make_activations(Lgu).to(dev)
+    prep_gu, gemm_gu, GU = layer_times(Lgu, Xgu, wl.make_weights(Lgu).to(dev), Lgu.had_block)
+    H = torch.empty((2048, 14336), dtype=torch.float16, device=dev)
+    silu = _time_ms(lambda: rrs.silu_mul(GU, H=H))
+    rrs.silu_mul(GU, H=H)
+    permd = rrs.calibrate_perm(H[:512], Ld.had_block)
+    qWd, swd = rrs.prepare_weights(wl.make_weights(Ld).to(dev), permd, Ld.had_block)
+    qXd = torch.empty((Ld.M, Ld.K // 2), dtype=torch.uint8, device=dev)
+    sd = torch.empty(Ld.K // Ld.G, dtype=torch.float32, device=dev)
+    std = torch.empty(Ld.M, dtype=torch.float32, device=dev)
+    Yd = torch.empty((Ld.M, Ld.N), dtype=torch.float32, device=dev)
+    wsd = rrs.make_workspace(Ld.M, Ld.N, Ld.K, Ld.G, Ld.had_block, device=dev)
+    prep_d = _time_ms(lambda: rrs.smooth_quant(H, permd, Ld.G, Ld.had_block, qX=qXd, s=sd, scale_t=std, ws=wsd))
+    gemm_d = _time_ms(lambda: rrs.w4a4_gemm(qXd, sd, std, qWd, swd, Ld.G, Y=Yd, ws=wsd, flags=rrs.WS_HOLDS_A8))
+    rrs.check_workspace(wsd)
+    total = prep_gu + gemm_gu + silu + prep_d + gemm_d
+    out["mlp_block"] = {"M": 2048, "K": 4096, "F": 14336, "G": 128,
+                        "us": {"gateup_prep": round(prep_gu * 1e3, 2), "gateup_gemm": round(gemm_gu * 1e3, 2),
+                               "silu_mul": round(silu * 1e3, 2), "down_prep": round(prep_d * 1e3, 2),
+                               "down_gemm": round(gemm_d * 1e3, 2), "total": round(total * 1e3, 2)},
+                        "silu_mul_GBps": round(2048 * 14336 * 10 / (silu * 1e-3) / 1e9, 1),
+                        "TOPS": round((Lgu.ops + Ld.ops) / (total * 1e-3) / 1e12, 1)}
+    del Xgu, GU, H
+    torch.cuda.empty_cache()
+
     names = ["llama3_8b_down", "llama3_70b_qo", "llama3_70b_gateup", "llama3_70b_down",
              "llama3_70b_qo_decode_m1", "llama3_70b_qo_decode_m8", "llama3_70b_qo_decode_m16",
              "llama3_70b_gateup_decode_m1", "llama3_70b_gateup_decode_m16",
