@@ -32,7 +32,7 @@ enum PrepMode : int { kQuant = 0, kGroupMax = 1, kChannelMax = 2 };
 
 // Swizzled word address of element `idx` in the fp32 row buffer: the 16-byte
 // chunk index (bits 2..4) is XORed with bits e..e+2 (e = log2 E >= 5), which makes both the
-// round-1 vector stores (each thread a contiguous run of E elements) and the
+// first-round vector stores (each thread a contiguous run of E elements) and the
 // later strided scalar accesses bank-conflict free.
 template <int LOGE>
 __device__ __forceinline__ int swz(int idx) {
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(MAXT) prep_kernel(PrepArgs p) {
     const int al = L - (nrounds - 1) * LOGE < LOGE ? L - (nrounds - 1) * LOGE : LOGE;
 
     // Per-thread gather addresses for the outputs j in [t*E, t*E + E) (kQuant).
-    constexpr int CH = E >= 8 ? E / 8 : 1;     // 16-byte fp16 chunks per thread in round 1
+    constexpr int CH = E >= 8 ? E / 8 : 1;     // 16-byte fp16 chunks per thread in the first round
     constexpr int EG = (MODE == kQuant) ? E / 2 : 1;
     uint32_t gaddr[EG];
     float d = 1.0f;
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(MAXT) prep_kernel(PrepArgs p) {
         named_bar(bar_id, T);
         const int tl = opaque(t);
 
-        // ---- round 1: E contiguous elements from the staging buffer.
+        // ---- first round: E contiguous elements from the staging buffer.
         float v[E];
         {
             const __half* st = stage0 + (size_t)sb * K;
