@@ -29,8 +29,13 @@ MUTATIONS = [
 ]
 
 
+PIN_SUITES = ["test_oracle_pins.py", "test_oracle_golden.py"]
+
+
+@pytest.mark.parametrize("suite", PIN_SUITES)
 @pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_pins_fail_on_planted_mistake(tmp_path, name, old, new):
+def test_pins_fail_on_planted_mistake(tmp_path, name, old, new, suite):
+    """Both the pin suite and the hand-worked example, each on its own, catch every mistake."""
     src = open(ob.SRC).read()
     assert src.count(old) == 1, f"mutation anchor not found for {name}"
     mut = tmp_path / "mut.c"
@@ -39,6 +44,6 @@ def test_pins_fail_on_planted_mistake(tmp_path, name, old, new):
     subprocess.check_call(["gcc", *ob.CFLAGS, str(mut), "-o", str(lib), "-lm"])
     env = dict(os.environ, RRS_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", suite)],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutation '{name}':\n{r.stdout[-2000:]}"
