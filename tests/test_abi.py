@@ -93,6 +93,23 @@ def test_argument_checks_fail_before_any_launch(L):
     assert len(L.rrs_last_error_string()) > 0
 
 
+def test_next_row_entry_points_check_arguments_before_any_launch(L):
+    ok = _fake(0x10000)
+    mis = _fake(0x10004)
+    # rrs_silu_mul(GU, M, F, H, stream)
+    assert L.rrs_silu_mul(None, 4, 8, ok, None) == 1
+    assert L.rrs_silu_mul(ok, 4, 8, None, None) == 1
+    assert L.rrs_silu_mul(mis, 4, 8, ok, None) == 1
+    assert b"aligned" in L.rrs_last_error_string()
+    assert L.rrs_silu_mul(ok, 0, 8, ok, None) == 1
+    assert L.rrs_silu_mul(ok, 4, 0, ok, None) == 1
+    # rrs_expand_weights(qW, N, K, qW8, stream)
+    assert L.rrs_expand_weights(None, 16, 256, ok, None) == 1
+    assert L.rrs_expand_weights(ok, 16, 256, mis, None) == 1
+    assert L.rrs_expand_weights(ok, 0, 256, ok, None) == 1
+    assert L.rrs_expand_weights(ok, 16, 200, ok, None) == 2     # K % 128 != 0: unsupported
+
+
 def test_binding_shape_checks_without_gpu():
     import torch
     import activation_smoothing_b200 as rrs
