@@ -212,3 +212,22 @@ def y_tolerance_ok(Y_gpu: np.ndarray, Y_orc: np.ndarray, bound: np.ndarray,
     |dY| <= rel*|Y| + 2^-20 * sum_g |s_g P_g| scale_t scale_w."""
     d = np.abs(Y_gpu.astype(np.float64) - Y_orc.astype(np.float64))
     return d <= rel * np.abs(Y_orc.astype(np.float64)) + (2.0 ** -20) * bound
+
+
+def silu_mul(GU) -> np.ndarray:
+    """The step between the two linears of a gated feed-forward block:
+    H = silu(gate) * up, with gate = GU[:, :F] and up = GU[:, F:] of the fused gate/up
+    projection's output, and silu(g) = g / (1 + exp(-g)).
+
+    The block is the feed-forward block of the LLaMA models the pages evaluate
+    (Rotated Runtime Smooth summary page, "Key results").  Its down projection takes an
+    online Hadamard rotation of its input ("Understanding LLM Quantization through
+    Activation-Guided Compensation and Orthogonal Residuals", Sec. 4.6).  Computed
+    in fp64, saturated to the fp16 range +-65504, and rounded once to fp16 (round half
+    to even): the down projection's fp16 activations.
+    """
+    gu = np.asarray(GU.detach().cpu().numpy() if hasattr(GU, "numpy") else GU, np.float64)
+    F = gu.shape[1] // 2
+    g, u = gu[:, :F], gu[:, F:]
+    h = g / (1.0 + np.exp(-g)) * u
+    return np.clip(h, -65504.0, 65504.0).astype(np.float16)
