@@ -165,7 +165,9 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t *qX, const uint8_t *qW, in
  * of N * K / 2) and makes the GEMM faster where it is compute-bound (prefill;
  * pass RRS_W_EXPANDED).  qW packed [N, K/2] as rrs_prepare_weights writes it;
  * qW8 [N, K] device, caller-owned, 16-byte aligned.  K as for rrs_w4a4_gemm.
- * Asynchronous on `stream`. */
+ * Asynchronous on `stream`.  Errors: RRS_ERR_INVALID_ARG for a null or misaligned
+ * pointer or N < 1; RRS_ERR_UNSUPPORTED for K % 128 != 0; RRS_ERR_CUDA if the launch
+ * fails. */
 rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, int8_t *qW8, rrs_stream_t stream);
 
 /* Gated-MLP step between two RRS linears (summary page "Key results": the method is
@@ -175,7 +177,8 @@ rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, int8_t *qW8, rrs_
  * output of the fused gate/up projection whose weight rows are [W_gate; W_up]; H fp16
  * [M, F], the down projection's X.  Both device, caller-owned, 16-byte aligned.  The
  * pages fix no activation function; SiLU is that of the LLaMA models they evaluate.
- * Asynchronous on `stream`. */
+ * Asynchronous on `stream`.  Errors: RRS_ERR_INVALID_ARG for a null or misaligned
+ * pointer or M, F < 1; RRS_ERR_CUDA if the launch fails. */
 rrs_status rrs_silu_mul(const float *GU, int M, int F, void *H, rrs_stream_t stream);
 
 /* Calibration statistic for the reorder index: cmax[k] = max_t |X_rot[t][k]|
