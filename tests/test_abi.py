@@ -118,6 +118,34 @@ def test_binding_shape_checks_without_gpu():
         rrs.smooth_quant(X, torch.arange(256, dtype=torch.int32), 128, 256)   # host tensors rejected
 
 
+def test_binding_flag_and_dtype_inference_without_gpu():
+    import torch
+    from activation_smoothing_b200 import _binding as b
+    assert b._y_flags(None, 0) == 0
+    assert b._y_flags(torch.empty(2, 2, dtype=torch.float32), b.WS_HOLDS_A8) == b.WS_HOLDS_A8
+    assert b._y_flags(torch.empty(2, 2, dtype=torch.bfloat16), 0) == b.Y_BF16
+    assert b._y_dtype(b.Y_BF16 | b.W_EXPANDED) == torch.bfloat16
+    assert b._y_dtype(b.W_EXPANDED) == torch.float32
+    # packed weights are uint8 [N, K/2]; expanded ones int8 [N, K]; host tensors are refused
+    with pytest.raises(TypeError):
+        b._need_weights(torch.zeros(4, 64, dtype=torch.int8), 4, 128, 0)
+    with pytest.raises(TypeError):
+        b._need_weights(torch.zeros(4, 128, dtype=torch.uint8), 4, 128, b.W_EXPANDED)
+    with pytest.raises(ValueError):
+        b._need_weights(torch.zeros(4, 64, dtype=torch.uint8), 4, 128, 0)
+    with pytest.raises(ValueError):
+        b._need_weights(torch.zeros(4, 128, dtype=torch.int8), 4, 128, b.W_EXPANDED)
+
+
+def test_next_row_bindings_refuse_host_tensors():
+    import torch
+    import activation_smoothing_b200 as rrs
+    with pytest.raises((TypeError, ValueError)):
+        rrs.silu_mul(torch.zeros(4, 16, dtype=torch.float32))
+    with pytest.raises((TypeError, ValueError)):
+        rrs.expand_weights(torch.zeros(4, 64, dtype=torch.uint8))
+
+
 def test_product_never_imports_the_oracle():
     pkg = os.path.join(ROOT, "activation_smoothing_b200")
     for dirpath, _, files in os.walk(pkg):
