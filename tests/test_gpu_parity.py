@@ -430,3 +430,16 @@ def test_markstein_division_matches_ieee(rrs):
     # and the IEEE division itself is the correctly rounded quotient (checked in double)
     ref = (a.astype(np.float64) / b.astype(np.float64)).astype(np.float32)
     assert np.array_equal(qi, ref)
+
+
+@pytest.mark.parametrize("name", ["llama3_70b_qo", "llama3_70b_gateup", "llama3_70b_down"])
+def test_llama3_70b_prefill_layers(rrs, name):
+    """70B prefill layers at full size (M=4096; K, N and the Hadamard blocks as defined):
+    every code and scale bit-exact, Y on sampled rows (the largest token scales, the first
+    and last rows, and random ones) within tolerance, packed and expanded weights
+    bit-identical."""
+    L = wl.LAYERS[name]
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = wl.random_perm(L.K, 5)
+    _, _, _, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
+    run_layer(rrs, X, W, perm, L.G, L.had_block, rows=_sample_rows(L.M, ost, k=8))
