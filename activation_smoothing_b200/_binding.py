@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         "rrs_workspace_size": ([I, I, I, I, I, U], Z),
         "rrs_prepare_weights": ([P, I, I, I, P, P, P, U, P], I),
         "rrs_smooth_quant": ([P, I, I, I, I, P, P, P, P, P, Z, U, P], I),
+        "rrs_group_max": ([P, I, I, I, I, P, P, P, Z, U, P], I),
+        "rrs_smooth_quant_scaled": ([P, I, I, I, I, P, P, P, P, P, Z, U, P], I),
         "rrs_w4a4_gemm": ([P, P, P, P, P, I, I, I, I, P, P, Z, U, P], I),
         "rrs_linear": ([P, P, P, P, I, I, I, I, I, P, P, P, P, P, Z, U, P], I),
         "rrs_linear_from_host": ([P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, Z, U, P], I),
@@ -151,6 +153,36 @@ def smooth_quant(X: torch.Tensor, perm: torch.Tensor, G: int, had_block: int, fl
     return qX, s, scale_t
 
 
+def group_max(X: torch.Tensor, perm: torch.Tensor, G: int, had_block: int, flags: int = 0,
+              s: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pass A of the activation path: s fp32 [K/G] = per-group max |X'| over these tokens."""
+    M, K = X.shape
+    _need(X, "X", torch.float16, (M, K))
+    _need(perm, "perm", torch.int32, (K,))
+    s = torch.empty(max(K // G, 1), dtype=torch.float32, device=X.device) if s is None else s
+    ws = make_workspace(M, 0, K, G, had_block, flags, X.device) if ws is None else ws
+    _check(lib().rrs_group_max(_ptr(X), M, K, G, had_block, _ptr(perm), _ptr(s), _ptr(ws), ws.numel(), flags,
+                               _stream(stream)))
+    return s
+
+
+def smooth_quant_scaled(X: torch.Tensor, perm: torch.Tensor, s: torch.Tensor, G: int, had_block: int,
+                        flags: int = 0, qX: Optional[torch.Tensor] = None, scale_t: Optional[torch.Tensor] = None,
+                        ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Pass B: (qX uint8 [M, K/2], scale_t fp32 [M]) with the given group scales s [K/G]."""
+    M, K = X.shape
+    _need(X, "X", torch.float16, (M, K))
+    _need(perm, "perm", torch.int32, (K,))
+    _need(s, "s", torch.float32, (K // G,))
+    dev = X.device
+    qX = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if qX is None else qX
+    scale_t = torch.empty(M, dtype=torch.float32, device=dev) if scale_t is None else scale_t
+    ws = make_workspace(M, 0, K, G, had_block, flags, dev) if ws is None else ws
+    _check(lib().rrs_smooth_quant_scaled(_ptr(X), M, K, G, had_block, _ptr(perm), _ptr(s), _ptr(qX), _ptr(scale_t),
+                                         _ptr(ws), ws.numel(), flags, _stream(stream)))
+    return qX, scale_t
+
+
 def _y_flags(Y: Optional[torch.Tensor], flags: int) -> int:
     """A bf16 Y selects the bf16 output (RRS_Y_BF16)."""
     if Y is not None and Y.dtype == torch.bfloat16:
@@ -164,7 +196,7 @@ def _y_dtype(flags: int) -> torch.dtype:
 
 def _need_weights(qW: torch.Tensor, N: int, K: int, flags: int):
     if flags & W_EXPANDED:
-        _need(qW, "qW", torch.int8, (N, K))
+        _need(qW, "qW", torch.float8_e4m3fn, (N, K))
     else:
         _need(qW, "qW", torch.uint8, (N, K // 2))
 
@@ -173,8 +205,8 @@ def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torc
               scale_w: torch.Tensor, G: int, Y: Optional[torch.Tensor] = None,
               ws: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
     """Group-scaled W4A4 GEMM -> Y fp32 [M, N].  flags=WS_HOLDS_A8 when ``ws`` is the
-    workspace the preceding smooth_quant of this qX wrote (skips re-expanding qX);
-    W_EXPANDED when ``qW`` is the int8 operand from expand_weights."""
+    workspace the preceding smooth_quant of this qX wrote (with the same W_EXPANDED bit;
+    skips re-expanding qX); W_EXPANDED when ``qW`` is the e4m3 operand from expand_weights."""
     M, K2 = qX.shape
     N = qW.shape[0]
     K = 2 * K2
@@ -269,13 +301,13 @@ def silu_mul(GU: torch.Tensor, H: Optional[torch.Tensor] = None, stream=None) ->
 
 
 def expand_weights(qW: torch.Tensor, qW8: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Int8 tensor-core operand [N, K] (16 q, GEMM k order) from packed INT4 weights [N, K/2];
-    pass it with flags=W_EXPANDED."""
+    """The INT4 weight codes one per byte as e4m3 numbers [N, K] (natural k order; every
+    code is exact in e4m3) from packed INT4 weights [N, K/2]; pass it with flags=W_EXPANDED."""
     N, K2 = qW.shape
     K = 2 * K2
     _need(qW, "qW", torch.uint8, (N, K2))
-    qW8 = torch.empty((N, K), dtype=torch.int8, device=qW.device) if qW8 is None else qW8
-    _need(qW8, "qW8", torch.int8, (N, K))
+    qW8 = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=qW.device) if qW8 is None else qW8
+    _need(qW8, "qW8", torch.float8_e4m3fn, (N, K))
     _check(lib().rrs_expand_weights(_ptr(qW), N, K, _ptr(qW8), _stream(stream)))
     return qW8
 

@@ -41,14 +41,23 @@ constexpr size_t kHeaderBytes = 256;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace layout: [header 256 B: error word] [int8 activation operand, M*K]
-// [fp32 reordered activations X', M*K*4, fast path only].
+// Workspace layout: [header 256 B: error word at 0, grid-barrier words at 64]
+// [activation operand for the GEMM, M*K bytes] [per-CTA group maxima of the
+// activation kernel: one row of K/128 floats per CTA, fast path only].  For
+// M <= 16 the space after the operand also takes the GEMM's split-k partial
+// sums (the activation kernel's table is dead by then).
+constexpr size_t kBarrierOffset = 64;
+constexpr int kMaxPartialRows = 1024;
 size_t ws_a8_offset() { return kHeaderBytes; }
-size_t ws_scratch_offset(int M, int K) { return kHeaderBytes + align256((size_t)M * K); }
 size_t ws_bytes_gemm(int M, int K) { return kHeaderBytes + align256((size_t)M * K); }
+int ws_partial_rows(int M, int K) {
+    const int R = rrs::prep_fast_rows_per_cta(K);
+    const int rows = (M + R - 1) / R;
+    return rows < kMaxPartialRows ? rows : kMaxPartialRows;
+}
 size_t ws_bytes_full(int M, int K, int n) {
     size_t b = ws_bytes_gemm(M, K);
-    if (rrs::prep_fast_supported(K, n)) b += align256(rrs::prep_fast_scratch_bytes(M, K));
+    if (rrs::prep_fast_supported(K, n)) b += align256((size_t)ws_partial_rows(M, K) * (K / 128) * 4);
     return b;
 }
 
@@ -93,8 +102,11 @@ rrs_status check_ws(void* ws, size_t ws_bytes, size_t need) {
     return RRS_OK;
 }
 
+// phase 3: group maxima then quantisation (rrs_smooth_quant); 1: group maxima
+// only (pass A, writes s); 2: quantisation with the caller's s (pass B).
 rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float c_n, const int32_t* perm,
-                               uint8_t* qX, float* s, float* scale_t, void* ws, unsigned flags, cudaStream_t st) {
+                               uint8_t* qX, float* s, float* scale_t, void* ws, unsigned flags, cudaStream_t st,
+                               int phase = 3) {
     const int unit = (flags & RRS_FORCE_UNIT_SCALES) ? 1 : 0;
     int8_t* qX8 = reinterpret_cast<int8_t*>(static_cast<unsigned char*>(ws) + ws_a8_offset());
     if (rrs::prep_fast_supported(K, n)) {
@@ -111,7 +123,12 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
         pf.qX = qX;
         pf.qX8 = qX8;
         pf.scale_t = scale_t;
-        pf.scratch = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + ws_scratch_offset(M, K));
+        pf.phase = phase;
+        pf.a_e4m3 = (flags & RRS_W_EXPANDED) != 0;
+        pf.partial = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + ws_bytes_gemm(M, K));
+        pf.partial_rows = ws_partial_rows(M, K);
+        pf.gbar = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kBarrierOffset);
+        pf.err = reinterpret_cast<uint32_t*>(ws);
         cudaError_t e = rrs::launch_prep_fast(pf, st);
         if (e != cudaSuccess) return cuda_fail(e, "rotation/quantise kernels");
         return RRS_OK;
@@ -125,7 +142,7 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
     pl.G = G;
     pl.c_n = c_n;
     pl.perm = perm;
-    if (!unit) {
+    if (!unit && (phase & 1)) {
         cudaError_t e = cudaMemsetAsync(s, 0, sizeof(float) * (size_t)(K / G), st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(s)");
         pl.mode = 1;
@@ -133,6 +150,7 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
         e = rrs::launch_prep(pl, st);
         if (e != cudaSuccess) return cuda_fail(e, "group-max kernel");
     }
+    if (!(phase & 2)) return RRS_OK;
     pl.mode = 0;
     pl.max_out = nullptr;
     pl.unit_scales = unit;
@@ -142,7 +160,8 @@ rrs_status launch_smooth_quant(const void* X, int M, int K, int G, int n, float 
     pl.s_unit_out = unit ? s : nullptr;
     cudaError_t e = rrs::launch_prep(pl, st);
     if (e != cudaSuccess) return cuda_fail(e, "quantise kernel");
-    e = rrs::launch_expand(qX, qX8, M, K, st);
+    e = (flags & RRS_W_EXPANDED) ? rrs::launch_expand_e4m3(qX, reinterpret_cast<uint8_t*>(qX8), M, K, st)
+                                 : rrs::launch_expand(qX, qX8, M, K, st);
     if (e != cudaSuccess) return cuda_fail(e, "expand kernel");
     return RRS_OK;
 }
@@ -151,6 +170,33 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
                                const float* scale_w, int M, int N, int K, int G, float* Y, int32_t* P,
                                void* ws, size_t ws_bytes, unsigned flags, cudaStream_t st) {
     int8_t* qX8 = reinterpret_cast<int8_t*>(static_cast<unsigned char*>(ws) + ws_a8_offset());
+    if (flags & RRS_W_EXPANDED) {
+        // fp8 operands: e4m3 activation codes in the workspace, e4m3 weight codes
+        if (!(flags & RRS_WS_HOLDS_A8)) {
+            cudaError_t e = rrs::launch_expand_e4m3(qX, reinterpret_cast<uint8_t*>(qX8), M, K, st);
+            if (e != cudaSuccess) return cuda_fail(e, "expand kernel");
+        }
+        rrs::GemmF8Launch gf{};
+        gf.A = qX8;
+        gf.B = qW;
+        gf.s = s;
+        gf.scale_t = scale_t;
+        gf.scale_w = scale_w;
+        gf.M = M;
+        gf.N = N;
+        gf.K = K;
+        gf.G = G;
+        gf.PB = rrs::promotion_block(G);
+        gf.Y = Y;
+        gf.P = P;
+        gf.err = reinterpret_cast<uint32_t*>(ws);
+        gf.y_bf16 = P == nullptr && (flags & RRS_Y_BF16) != 0;
+        gf.bn = 0;
+        gf.stream = st;
+        cudaError_t e = rrs::launch_gemm_f8(gf);
+        if (e != cudaSuccess) return cuda_fail(e, "GEMM kernel");
+        return RRS_OK;
+    }
     if (!(flags & RRS_WS_HOLDS_A8)) {
         cudaError_t e = rrs::launch_expand(qX, qX8, M, K, st);
         if (e != cudaSuccess) return cuda_fail(e, "expand kernel");
@@ -168,7 +214,6 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
     gl.Y = Y;
     gl.P = P;
     gl.err = reinterpret_cast<uint32_t*>(ws);
-    gl.w_expanded = (flags & RRS_W_EXPANDED) != 0;
     gl.y_bf16 = P == nullptr && (flags & RRS_Y_BF16) != 0;
     // Room after the int8 operand (the activation scratch, dead once the
     // activation kernels have run) takes split-k partial sums for small M.
@@ -196,27 +241,60 @@ constexpr size_t kNoAllocBytes = kHeaderBytes + kNoAllocMaxElems + kNoAllocMaxEl
 static __device__ __align__(256) unsigned char g_noalloc_ws[kNoAllocBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_ws on the current device (looked up on first use).
+// Device address of g_noalloc_ws on the current device.  Looked up on every
+// call (cheap once the module is loaded), so that it stays right after the
+// device's context is reset and the module reloaded.
 rrs_status noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) return fail(RRS_ERR_UNSUPPORTED, "device index %d out of range", dev);
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_ws);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    *out = p;
     return RRS_OK;
 }
 }  // namespace
+
+namespace rrs {
+
+int device_sm_count() {
+    static int cached[16] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 16) {
+        int n = 148;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        return n;
+    }
+    if (cached[dev] == 0) {
+        int n = 148;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+cudaError_t kernel_setup(const void* kern, int threads, size_t smem, KernelSetup& cache, int* occ_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cacheable = dev >= 0 && dev < 16;
+    if (cacheable && cache.attr[dev] && cache.occ[dev] > 0) {
+        *occ_out = cache.occ[dev];
+        return cudaSuccess;
+    }
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (cacheable) {
+        cache.attr[dev] = true;
+        cache.occ[dev] = occ;
+    }
+    *occ_out = occ;
+    return cudaSuccess;
+}
+
+}  // namespace rrs
 
 extern "C" {
 
@@ -285,6 +363,58 @@ rrs_status rrs_smooth_quant(const void* X, int M, int K, int G, int had_block, c
     if (r != RRS_OK) return r;
     return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, s, scale_t, ws, flags,
                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+rrs_status rrs_group_max(const void* X, int M, int K, int G, int had_block, const int32_t* perm, float* s,
+                         void* ws, size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(X);
+    RRS_REQUIRE_PTR(perm);
+    RRS_REQUIRE_PTR(s);
+    if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    r = check_ws(ws, ws_bytes, ws_bytes_full(M, K, n));
+    if (r != RRS_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (flags & RRS_FORCE_UNIT_SCALES) {
+        // no smoothing: every scale is 1
+        cudaError_t e = rrs::launch_fill(s, K / G, 1.0f, st);
+        if (e != cudaSuccess) return cuda_fail(e, "fill kernel");
+        return RRS_OK;
+    }
+    return launch_smooth_quant(X, M, K, G, n, c_n, perm, nullptr, s, nullptr, ws, flags & ~RRS_W_EXPANDED, st, 1);
+}
+
+rrs_status rrs_smooth_quant_scaled(const void* X, int M, int K, int G, int had_block, const int32_t* perm,
+                                   const float* s, uint8_t* qX, float* scale_t, void* ws, size_t ws_bytes,
+                                   unsigned flags, rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(X);
+    RRS_REQUIRE_PTR(perm);
+    RRS_REQUIRE_PTR(s);
+    RRS_REQUIRE_PTR(qX);
+    RRS_REQUIRE_PTR(scale_t);
+    if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
+    rrs_status r = check_K(K);
+    if (r != RRS_OK) return r;
+    r = check_G(K, G);
+    if (r != RRS_OK) return r;
+    int n;
+    float c_n;
+    r = check_hadamard(K, had_block, flags, &n, &c_n);
+    if (r != RRS_OK) return r;
+    r = check_ws(ws, ws_bytes, ws_bytes_full(M, K, n));
+    if (r != RRS_OK) return r;
+    if (flags & RRS_FORCE_UNIT_SCALES)
+        return fail(RRS_ERR_INVALID_ARG, "rrs_smooth_quant_scaled takes its scales from s; RRS_FORCE_UNIT_SCALES "
+                                         "does not apply (pass s filled with 1 instead)");
+    return launch_smooth_quant(X, M, K, G, n, c_n, perm, qX, const_cast<float*>(s), scale_t, ws, flags,
+                               reinterpret_cast<cudaStream_t>(stream), 2);
 }
 
 rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
@@ -369,7 +499,8 @@ rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, int8_t* qW8, rrs_
     if (N < 1) return fail(RRS_ERR_INVALID_ARG, "N = %d", N);
     rrs_status r = check_K(K);
     if (r != RRS_OK) return r;
-    cudaError_t e = rrs::launch_expand_weights(qW, qW8, N, K, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = rrs::launch_expand_e4m3(qW, reinterpret_cast<uint8_t*>(qW8), N, K,
+                                            reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "expand_weights kernel");
     return RRS_OK;
 }

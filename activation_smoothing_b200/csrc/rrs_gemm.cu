@@ -26,11 +26,11 @@
 //
 // Exact promotion: the weight operand holds 16 q, so a group's int32 sum is
 // 16 * P_g with |16 P_g| <= 16 * 64 * 4096 = 2^22 for groups of up to 4096 k;
-// its int32 -> fp32 conversion is then exact.  Longer groups are promoted in
-// 4096-wide blocks with the same s_g.
+// its int32 -> fp32 conversion is then exact.
 //
-// A second kernel (gemm_w8_kernel, below) takes the weights already expanded
-// to that int8 operand and needs no unpack warps.
+// Longer groups are promoted in blocks of up to 4096 k that divide the group
+// (promotion_block).  Weights expanded to one code per byte take the fp8
+// kernel of rrs_gemm_f8.cu instead.
 //
 // k order: inside each 32-wide k chunk both operands store the codes in the
 // order 0,2,4,6,1,3,5,7, 8,10,... (what a nibble mask produces); the integer
@@ -470,163 +470,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-// ------------------------------------------------------------------------
-// Variant for weights stored as the expanded int8 operand (16 q in the GEMM's
-// k order, written once by rrs_expand_weights).  Nothing is unpacked, so the
-// CTA needs no unpack warps; warps 0, 2 and 3 instead each feed the stage ring.
-// A bulk copy's round trip is not overlapped with the next copy a warp issues,
-// so one producer warp keeps one stage in flight and three keep three: stage
-// `it` is loaded by producer it % 3, its activation tile and weight tile by
-// lanes 0 and 1 of that warp in one instruction, onto one barrier.
-namespace w8 {
-constexpr int NST = 5;                        // stages of activation + weight tiles (40 KB each)
-constexpr int NPROD = 3;                      // producer warps
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + NST * A_BYTES;
-constexpr int OFF_BAR = OFF_B + NST * B8_BYTES;
-constexpr int OFF_S = OFF_BAR + 1024;
-constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
-static_assert(SMEM <= 227 * 1024, "shared memory budget");
-static_assert(OFF_B % 1024 == 0 && B8_BYTES % 1024 == 0, "128-byte-swizzled tiles need 1024-byte alignment");
-}  // namespace w8
-
-template <bool DEBUG_P, bool SPLIT, bool YBF16>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
-    extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + w8::OFF_BAR);
-    uint64_t* empty = full + w8::NST;
-    uint64_t* tfull = empty + w8::NST;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* done = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-    float* s_sm = reinterpret_cast<float*>(smem + w8::OFF_S);
-    volatile int* abortv = abort_flag;
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int KB = g.K / BK;
-    const int NPB = g.K / g.PB;
-    const int kb_per_pb = g.PB / BK;
-    const int GS = SPLIT ? g.S : 1;
-    const int KBS = KB / GS;
-    const int nmb = (g.M + BM - 1) / BM;
-    const int nnb = (g.N + BN - 1) / BN;
-    const int ntiles = nmb * nnb;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < w8::NST; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], EPI_WARPS);
-        }
-        mbar_init(done, 1);
-        *abort_flag = 0;
-        mbar_fence_init();
-    }
-    if (!DEBUG_P) {
-        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
-    }
-    if (warp == 2) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0 || warp == 2 || warp == 3) {
-        // -------------------------------------------------------- TMA
-        const uint32_t p = warp == 0 ? 0u : (uint32_t)(warp - 1);
-        const int nwork = ntiles * GS;
-        const uint32_t my_items = blockIdx.x < (unsigned)nwork ? (nwork - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-        const uint32_t total = my_items * KBS;
-        uint32_t last = 0xFFFFFFFFu;          // last stage this warp loaded
-        bool ok = true;
-        for (uint32_t it = p; it < total; it += w8::NPROD) {
-            const int st = (int)(it % w8::NST);
-            uint32_t free = 1;
-            if (lane == 0)
-                free = mbar_wait_bounded<true>(&empty[st], ((it / w8::NST) & 1u) ^ 1u, abortv, g.err, kErrGemmTimeout,
-                                               g.limit_ns) ? 1u : 0u;
-            if (!__shfl_sync(0xffffffffu, free, 0)) {
-                ok = false;
-                break;
-            }
-            const int w = blockIdx.x + (int)(it / KBS) * gridDim.x;
-            const int tile = w / GS;
-            const int kb = (w % GS) * KBS + (int)(it % KBS);
-            if (lane == 0) arrive_expect_tx(&full[st], A_BYTES + B8_BYTES);
-            __syncwarp();
-            if (lane < 2) {
-                unsigned char* dst = lane == 0 ? smem + w8::OFF_A + st * A_BYTES : smem + w8::OFF_B + st * B8_BYTES;
-                const CUtensorMap* map = lane == 0 ? &tmA : &tmB;
-                const int y = lane == 0 ? (tile % nmb) * BM : (tile / nmb) * BN;
-                tma_load_2d(dst, map, kb * BK, y, &full[st]);
-            }
-            __syncwarp();
-            last = it;
-        }
-        if (!ok && lane == 0 && last != 0xFFFFFFFFu) {
-            // let this warp's copies land before the CTA exits
-            volatile int no_abort = 0;
-            mbar_wait_bounded<true>(&full[last % w8::NST], (last / w8::NST) & 1u, &no_abort, nullptr, 0, g.limit_ns);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // -------------------------------------------------------- MMA
-            constexpr uint32_t idesc = idesc_i8(BM, BN);
-            uint32_t it = 0, gc = 0;
-            bool ok = true;
-            for (int w = blockIdx.x; w < ntiles * GS && ok; w += gridDim.x) {
-                for (int kb = 0; kb < KBS; ++kb, ++it) {
-                    const bool first = (kb % kb_per_pb) == 0;
-                    const bool lastk = (kb % kb_per_pb) == kb_per_pb - 1;
-                    const int buf = gc & 1;
-                    if (first && !(ok = mbar_wait_bounded<true>(&tempty[buf], (gc >> 1) & 1u, abortv, g.err,
-                                                                kErrGemmTimeout, g.limit_ns)))
-                        break;
-                    const int st = (int)(it % w8::NST);
-                    if (!(ok = mbar_wait_bounded<true>(&full[st], (it / w8::NST) & 1u, abortv, g.err,
-                                                       kErrGemmTimeout, g.limit_ns)))
-                        break;
-                    tc_fence_after();
-                    const uint32_t a_base = smem_u32(smem + w8::OFF_A + st * A_BYTES);
-                    const uint32_t b_base = smem_u32(smem + w8::OFF_B + st * B8_BYTES);
-                    const uint32_t d = tmem + (uint32_t)(buf * TMEM_BUF);
-#pragma unroll
-                    for (int k = 0; k < BK / 32; ++k)
-                        umma_i8(d, sdesc_k_sw128(a_base + 32 * k), sdesc_k_sw128(b_base + 32 * k), idesc,
-                                (first && k == 0) ? 0u : 1u);
-                    tc_commit(&empty[st]);
-                    if (lastk) {
-                        tc_commit(&tfull[buf]);
-                        ++gc;
-                    }
-                }
-            }
-            tc_commit(done);
-            volatile int no_abort = 0;
-            mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
-        }
-    } else {
-        epilogue_role<DEBUG_P, SPLIT, YBF16>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles * GS, nmb, NPB / GS);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 2) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
 // Y = (sum over splits of the partial sums, in split order) * scale_t * scale_w.
 // The partials already carry the factor 1/16, so the products are applied in
 // the order of the unsplit epilogue.
@@ -693,18 +536,20 @@ static bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint
 
 }  // namespace gemm
 
+int promotion_block(int G) {
+    int pb = G < gemm::MAX_PB ? G : gemm::MAX_PB;
+    pb -= pb % 128;
+    while (pb > 128 && G % pb != 0) pb -= 128;
+    return pb;
+}
+
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     using namespace gemm;
     CUtensorMap tmA, tmB;
     if (!make_map_u8(&tmA, gl.qX8, (uint64_t)gl.K, (uint64_t)gl.M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (gl.w_expanded) {
-        if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K, (uint64_t)gl.N, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-    } else if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K / 2, (uint64_t)gl.N, BK / 2, BN,
-                            CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    if (!make_map_u8(&tmB, gl.qW, (uint64_t)gl.K / 2, (uint64_t)gl.N, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    }
     Args a;
     a.s = gl.s;
     a.scale_t = gl.scale_t;
@@ -713,14 +558,12 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     a.N = gl.N;
     a.K = gl.K;
     a.G = gl.G;
-    a.PB = gl.G < MAX_PB ? gl.G : MAX_PB;
+    a.PB = promotion_block(gl.G);
     a.Y = gl.Y;
     a.P = gl.P;
     a.err = gl.err;
     a.limit_ns = kWaitLimitNs;
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = device_sm_count();
     const int ntiles = ((gl.M + BM - 1) / BM) * ((gl.N + BN - 1) / BN);
     // Few tiles (decode token counts): split k over whole promotion blocks so that
     // every SM streams weights, if the workspace has room for the partial sums.
@@ -736,16 +579,8 @@ cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream) {
     const int nwork = ntiles * S;
     const int grid = nwork < nsm ? nwork : nsm;
     cudaError_t e;
-    if (gl.w_expanded) {
-        // (with split k the bf16 rounding happens in splitk_reduce_kernel)
-        auto kern = gl.P     ? gemm_w8_kernel<true, false, false>
-                    : S > 1  ? gemm_w8_kernel<false, true, false>
-                    : a.ybf16 ? gemm_w8_kernel<false, false, true>
-                              : gemm_w8_kernel<false, false, false>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w8::SMEM);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, NTHREADS, w8::SMEM, stream>>>(tmA, tmB, a);
-    } else if (gl.P) {
+    // (with split k the bf16 rounding happens in splitk_reduce_kernel)
+    if (gl.P) {
         auto kern = gemm_kernel<true, false, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;

@@ -9,6 +9,19 @@
 
 namespace rrs {
 
+// Per-device launch facts, looked up once per device and kept: the number of
+// SMs, and for a kernel the dynamic shared memory attribute already set and
+// its occupancy.  Launch paths call these instead of querying the runtime on
+// every call (the queries cost more host time than a small kernel runs).
+int device_sm_count();
+// Sets the kernel's dynamic shared-memory limit (first call per device) and
+// returns blocks per SM for (threads, smem); `cache` is the kernel's own slot.
+struct KernelSetup {
+    int occ[16] = {0};
+    bool attr[16] = {false};
+};
+cudaError_t kernel_setup(const void* kern, int threads, size_t smem, KernelSetup& cache, int* occ_out);
+
 struct PrepLaunch {
     const void* X;          // fp16 [rows, K]
     int rows, K, n, G;
@@ -27,7 +40,7 @@ cudaError_t launch_prep(const PrepLaunch& pl, cudaStream_t stream);
 
 struct GemmLaunch {
     const int8_t* qX8;      // [M, K] int8 activation codes (k order of the fast prep / expand kernels)
-    const uint8_t* qW;      // [N, K/2] packed INT4 weights, or [N, K] int8 16 q when w_expanded
+    const uint8_t* qW;      // [N, K/2] packed INT4 weights
     const float* s;         // [K/G]
     const float* scale_t;   // [M]
     const float* scale_w;   // [N]
@@ -35,7 +48,6 @@ struct GemmLaunch {
     float* Y;               // [M, N] (null in debug mode)
     int32_t* P;             // [K/G, M, N] debug partials (null in normal mode)
     uint32_t* err;          // workspace error word
-    bool w_expanded;        // qW holds the expanded operand written by launch_expand_weights
     float* part;            // workspace room for split-k partial sums (may be null)
     size_t part_bytes;
     bool y_bf16;            // Y is bf16 [M, N] instead of fp32
@@ -46,30 +58,59 @@ struct GemmLaunch {
 constexpr int kSplitRoomMaxM = 16;
 constexpr int kSplitRoom = 16;
 
-// Fast activation path (K % 2048 == 0): rotation + reorder + group max into an
-// fp32 scratch, then smoothing + quantisation.
+// Fast activation path (K % 2048 == 0): one cooperative kernel, phase A (group
+// maxima -> s) and phase B (quantise with s), no M x K intermediate.
 struct PrepFastLaunch {
     const void* X;          // fp16 [rows, K]
     int rows, K, n, G;
     float c_n;
     const int32_t* perm;
     int unit_scales;
-    float* s;               // [K/G] output (max of |X'| per group, or 1)
+    int phase;              // 3: both phases; 1: phase A only (writes s); 2: phase B only (reads s)
+    float* s;               // [K/G]
     uint8_t* qX;            // [rows, K/2]
-    int8_t* qX8;            // [rows, K]
+    int8_t* qX8;            // [rows, K] GEMM operand or null: int8 codes (GEMM k order), or e4m3 (natural) if a_e4m3
     float* scale_t;         // [rows]
-    float* scratch;         // [rows, K] fp32
+    bool a_e4m3;            // write the fp8 GEMM operand instead of the int8 one
+    float* partial;         // per-CTA group maxima: partial_rows x K/G floats (workspace)
+    int partial_rows;       // capacity of that table in CTAs (caps the grid)
+    uint32_t* gbar;         // grid barrier words (workspace header, zero-filled)
+    uint32_t* err;          // workspace error word
 };
 
 bool prep_fast_supported(int K, int n);
-size_t prep_fast_scratch_bytes(int M, int K);
+int prep_fast_rows_per_cta(int K);
 cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t stream);
+// p[0..n) = v.
+cudaError_t launch_fill(float* p, int n, float v, cudaStream_t stream);
 // Packed INT4 rows -> int8 rows in the GEMM's k order.
 cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStream_t stream);
-// Packed INT4 weight rows -> int8 rows holding 16 q, in the same k order.
-cudaError_t launch_expand_weights(const uint8_t* qW, int8_t* qW8, int N, int K, cudaStream_t stream);
 
 cudaError_t launch_gemm(const GemmLaunch& gl, cudaStream_t stream);
+
+// Prefill GEMM on fp8 (e4m3) operands: both INT4 code sets stored one code per
+// byte as e4m3 numbers in natural k order (exact; see rrs_gemm_f8.cu).
+struct GemmF8Launch {
+    const void* A;          // e4m3 [M, K] activation codes
+    const void* B;          // e4m3 [N, K] weight codes
+    const float* s;         // [K/G]
+    const float* scale_t;   // [M]
+    const float* scale_w;   // [N]
+    int M, N, K, G, PB;     // PB: promotion block (a multiple of 128 dividing G, <= 4096)
+    void* Y;                // fp32 or bf16 [M, N] (null in debug mode)
+    int32_t* P;             // [K/G, M, N] debug partials (null in normal mode)
+    uint32_t* err;          // workspace error word
+    bool y_bf16;
+    int bn;                 // tile width 128 or 256; 0 = chosen from the shape
+    cudaStream_t stream;
+};
+cudaError_t launch_gemm_f8(const GemmF8Launch& gl);
+int gemm_f8_pick_bn(int M, int N, int nsm);
+// Packed INT4 rows [rows, K/2] -> e4m3 codes [rows, K], natural k order.
+cudaError_t launch_expand_e4m3(const uint8_t* q, uint8_t* out, int rows, int K, cudaStream_t stream);
+// Longest block of k, a multiple of 128 and at most 4096, that divides G: the
+// unit in which both GEMMs promote exact partial sums.
+int promotion_block(int G);
 // H fp16 [M, F] = silu(GU[:, :F]) * GU[:, F:], GU fp32 [M, 2F].
 cudaError_t launch_silu_mul(const float* GU, int M, int F, void* H, cudaStream_t stream);
 cudaError_t launch_divide_check(const float* a, const float* b, int n, float* q_fast, float* q_ieee,

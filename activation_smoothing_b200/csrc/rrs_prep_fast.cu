@@ -1,18 +1,26 @@
 // rrs_prep_fast.cu -- online activation path for K a multiple of 2048 (every
-// LLaMA projection shape): two kernels with an fp32 scratch between them.
+// LLaMA projection shape): one cooperative persistent kernel in two phases.
 //
-//   rot_gather_kernel   X (fp16) -> X' = reorder(rotate(X)) (fp32, scratch) and
-//                       s[g] = max over tokens and group channels |X'|
-//   smooth_quant_kernel X' -> qX (packed INT4), qX8 (int8 GEMM operand), scale_t
+//   phase A   X (fp16) -> Hadamard rotation of every row this CTA owns; the
+//             largest |X_rot| of each channel over those rows (registers), then
+//             through the reorder index the CTA's largest |X'| per group, into
+//             one row of a per-CTA table in the workspace
+//   barrier   a grid-wide barrier (bounded wait); every CTA then reduces the
+//             table: s[g] = max over all tokens and group channels of |X'|
+//   phase B   X again (an L2 hit) -> the same rotation bit for bit, reorder
+//             gather, division by s_g, per-token INT4 quantisation; writes qX
+//             (packed), scale_t and, if asked, the GEMM operand
 //
-// The scratch holds X' once (M*K*4 bytes), so the Hadamard transform runs once
-// per element; at the LLaMA-3-8B shapes the scratch (33.5 MB) stays in L2.
+// Nothing of size M x K passes between the phases: the rotation is recomputed
+// instead of stored.  The group max needs no gather in phase A: max over
+// tokens commutes with the reorder, and c_n * |v| is monotone in |v|, so
+// s_g = RN(c_n * max_{j in g} max_t |v_t[perm[j]]|) exactly.
 //
-// Work split: a team of T = K/64 threads (a multiple of 32) owns one row; each
-// thread holds 64 elements.  Rotation rounds: up to 6 butterfly stages on the
-// 64 registers (f32x2 packed add/sub for every stage but the first of a round),
-// an exchange through a swizzled fp32 row buffer, the next 6 stages (and a
-// third round for n = 8192).
+// Work split: a team of T = K/64 threads (a multiple of 32) owns one row at a
+// time; each thread holds 64 elements.  Rotation rounds: up to 6 butterfly
+// stages on the 64 registers (f32x2 packed add/sub for every stage but the
+// first of a round), an exchange through a swizzled fp32 row buffer, the next 6
+// stages (and a third round for n = 8192).
 //
 // Arithmetic is bit-identical to the library contract: stage order h = 1, 2, 4,
 // ... with (a + b, a - b); one multiply by c_n; IEEE division (computed with
@@ -105,151 +113,6 @@ __device__ __forceinline__ void rstore(const float2 (&v)[32], float* buf, int t,
     }
 }
 
-struct RotArgs {
-    const __half* X;     // [rows, K]
-    int rows, K, G;
-    float c_n;
-    const int32_t* perm; // [K]
-    float* xp;           // scratch [rows, K] fp32, thread-interleaved (see xp_offset)
-    uint32_t* smax;      // [K/G] fp32 bits, zeroed by the host
-};
-
-// Scratch layout of one row: the 64 reordered values of team thread t are 16
-// float4 at float4 index i*T + t (i = 0..15), so both the writes here and the
-// reads of smooth_quant_kernel are coalesced.
-__device__ __forceinline__ size_t xp_row(int r, int K) { return (size_t)r * K; }
-
-template <int L, int MAXT>
-__global__ void __launch_bounds__(MAXT) rot_gather_kernel(RotArgs p) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    constexpr int NR = (L <= LOGE) ? 1 : (L <= 2 * LOGE ? 2 : 3);
-    constexpr int A1 = L < LOGE ? L : LOGE;
-    constexpr int A2 = (L - LOGE) < LOGE ? (L - LOGE) : LOGE;
-    constexpr int A3 = L - 2 * LOGE;
-    const int K = p.K;
-    const int T = K / E;
-    const int R = blockDim.x / T;
-    const int team = threadIdx.x / T;
-    const int t = threadIdx.x % T;
-    float* rowbuf = reinterpret_cast<float*>(smem_raw) + (size_t)team * K;
-    __half* stage0 = reinterpret_cast<__half*>(reinterpret_cast<float*>(smem_raw) + (size_t)R * K) +
-                     (size_t)team * 2 * K;
-    const int bar_id = 1 + team;
-
-    // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
-    // perm is staged through shared memory: coalesced 16-byte global loads, and
-    // 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
-    // chunk reads below are bank-conflict free.
-    uint32_t gaddr[32];
-    {
-        int4* pst = reinterpret_cast<int4*>(smem_raw);
-        const int4* pg = reinterpret_cast<const int4*>(p.perm);
-        for (int c = threadIdx.x; c < K / 4; c += blockDim.x) pst[c ^ ((c >> 4) & 7)] = pg[c];
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int c = t * 16 + m;
-            const int4 v = pst[c ^ ((c >> 4) & 7)];
-            gaddr[2 * m] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
-            gaddr[2 * m + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
-        }
-        __syncthreads();   // the row buffers reuse this space
-    }
-    float tmax = 0.0f;
-
-    auto issue_row = [&](int r, int sb) {
-        const __half* src = p.X + (size_t)r * K;
-        __half* dst = stage0 + (size_t)sb * K;
-        for (int u = t; u < K / 8; u += T) {
-            const int owner = u >> 3;
-            const int c = u & 7;
-            cp_async16(dst + (size_t)(owner * 8 + (c ^ (owner & 7))) * 8, src + (size_t)u * 8);
-        }
-    };
-
-    const int stride = gridDim.x * R;
-    int r = blockIdx.x * R + team;
-    int it = 0;
-    if (r < p.rows) issue_row(r, 0);
-    cp_async_commit();
-    for (; r < p.rows; r += stride, ++it) {
-        const int sb = it & 1;
-        if (r + stride < p.rows) issue_row(r + stride, sb ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        named_bar(bar_id, T);
-        const int tl = opaque(t);
-
-        float2 v[32];
-        {
-            const __half* st = stage0 + (size_t)sb * K;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(st + (size_t)(tl * 8 + (c ^ (tl & 7))) * 8);
-                const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) v[c * 4 + q] = __half22float2(h2[q]);
-            }
-        }
-        stages<A1>(v);
-        if constexpr (NR >= 2) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2)
-                *reinterpret_cast<float4*>(rowbuf + swz(tl * E + 2 * i)) =
-                    make_float4(v[i].x, v[i].y, v[i + 1].x, v[i + 1].y);
-            named_bar(bar_id, T);
-            rload<LOGE, A2>(v, rowbuf, tl, T);
-            stages<A2>(v);
-        }
-        if constexpr (NR >= 3) {
-            rstore<LOGE, LOGE>(v, rowbuf, tl, T);
-            named_bar(bar_id, T);
-            rload<2 * LOGE, A3>(v, rowbuf, tl, T);
-            stages<A3>(v);
-        }
-        // X_rot = c_n * v, written in natural (swizzled) order for the gather.
-        const float2 c2 = make_float2(p.c_n, p.c_n);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], c2);
-        if constexpr (NR == 1) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2)
-                *reinterpret_cast<float4*>(rowbuf + swz(tl * E + 2 * i)) =
-                    make_float4(v[i].x, v[i].y, v[i + 1].x, v[i + 1].y);
-        } else if constexpr (NR == 2) {
-            rstore<LOGE, A2>(v, rowbuf, tl, T);
-        } else {
-            rstore<2 * LOGE, A3>(v, rowbuf, tl, T);
-        }
-        named_bar(bar_id, T);
-
-        // gather X'[j] = X_rot[perm[j]], track the group max, write the scratch
-        float4* dst = reinterpret_cast<float4*>(p.xp + xp_row(r, K));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t g0 = gaddr[2 * i], g1 = gaddr[2 * i + 1];
-            float4 o;
-            o.x = rowbuf[g0 & 0xFFFFu];
-            o.y = rowbuf[g0 >> 16];
-            o.z = rowbuf[g1 & 0xFFFFu];
-            o.w = rowbuf[g1 >> 16];
-            tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
-            dst[i * T + t] = o;
-        }
-        named_bar(bar_id, T);   // row buffer and staging free for the next row
-    }
-    cp_async_wait<0>();
-
-    // group max: G/64 consecutive threads share a group; reduce over aligned
-    // power-of-two segments of them, then one atomic per segment.
-    if (p.smax) {
-        const int gsz = p.G / E;
-        const int seg = (gsz & -gsz) < 32 ? (gsz & -gsz) : 32;
-        float m = tmax;
-        for (int o = seg >> 1; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if ((t % seg) == 0 && m > 0.0f) atomicMax(&p.smax[(t * E) / p.G], __float_as_uint(m));
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Division a / b for b > 0 by Markstein's method (P. Markstein, "Computation of
@@ -265,67 +128,300 @@ __device__ __forceinline__ float2 div_markstein(float2 a, float2 nb, float2 y) {
     return __ffma2_rn(r, y, q0);
 }
 
-struct QuantArgs {
-    const float* xp;     // scratch [rows, K] (thread-interleaved rows)
-    int rows, K, G;
-    int unit_scales;
-    const float* s;      // [K/G]
-    uint8_t* qX;         // [rows, K/2]
-    int8_t* qX8;         // [rows, K] int8 GEMM operand (k order permuted inside each 32-chunk)
-    float* scale_t;      // [rows]
-    float* s_unit_out;   // [K/G] written as 1 under unit scales (may be null)
-};
 
 // Gathers byte 0 of four words into one word: result byte i = byte 0 of w_i.
 __device__ __forceinline__ uint32_t low_bytes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
     return __byte_perm(__byte_perm(w0, w1, 0x0040), __byte_perm(w2, w3, 0x0040), 0x5410);
 }
 
-template <int MAXT>
-__global__ void __launch_bounds__(MAXT) smooth_quant_kernel(QuantArgs p) {
+// Two codes (integers in [-8, 7], exact in e4m3) -> two e4m3 bytes: lo in
+// the low byte, hi in the high byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+
+
+struct ActArgs {
+    const __half* X;     // [rows, K]
+    int rows, K, G, NG;
+    float c_n;
+    const int32_t* perm; // [K]
+    int phase;           // bit 0: phase A (group maxima -> s), bit 1: phase B (quantise with s)
+    int unit_scales;     // s := 1 (no phase A)
+    float* s;            // [NG]: written by phase A (CTA 0), read when phase B runs alone
+    uint8_t* qX;         // [rows, K/2]
+    uint8_t* a8;         // GEMM operand [rows, K] or null
+    int a8_mode;         // 1: int8 codes in the packed kernel's k order; 2: e4m3 codes, natural k order
+    float* scale_t;      // [rows]
+    float* partial;      // [gridDim.x, NG] per-CTA group maxima
+    uint32_t* gbar;      // grid barrier state: arrival count, generation (zero-filled before first use)
+    uint32_t* err;       // workspace error word
+    uint64_t limit_ns;
+};
+
+// Rows of one CTA for a given K (T = K/64 threads per row).
+__host__ __device__ constexpr int act_rows_per_cta(int K) { return (K / E) <= CTA ? CTA / (K / E) : 1; }
+// Shared memory: R fp32 row buffers, R double-buffered fp16 staging rows,
+// 256 words of group maxima / scales, R x 16 floats of row-max partials.
+__host__ __device__ constexpr size_t act_smem_bytes(int K) {
+    return (size_t)act_rows_per_cta(K) * K * 8 + 1024 + (size_t)act_rows_per_cta(K) * 64;
+}
+
+// Grid-wide barrier for a cooperative launch: sense reversal on two words
+// (arrival count, generation).  The last CTA to arrive resets the count and
+// advances the generation; the others wait for the generation to change, at
+// most limit_ns, then record a timeout in the error word and report failure.
+__device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t* err, uint64_t limit_ns) {
+    __shared__ int ok_s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        volatile uint32_t* vgen = gbar + 1;
+        const uint32_t gen = *vgen;
+        __threadfence();
+        const uint32_t old = atomicAdd(gbar, 1u);
+        if (old == gridDim.x - 1) {
+            atomicExch(gbar, 0u);
+            __threadfence();
+            atomicAdd(gbar + 1, 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t it = 0;
+            while (*vgen == gen) {
+                if ((++it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+                    atomicOr(err, kErrPrepTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        ok_s = ok;
+    }
+    __syncthreads();
+    return ok_s != 0;
+}
+
+// Loads the staged fp16 row into v and runs every butterfly stage of the
+// block Hadamard transform (no scaling).  On return v holds the elements in
+// the layout of the last round (see store_natural); the row buffer holds
+// intermediate values that only this thread's own positions will overwrite.
+template <int L>
+__device__ __forceinline__ void rotate_row(float2 (&v)[32], float* rowbuf, const __half* st, int tl, int T,
+                                           int bar_id) {
+    constexpr int NR = (L <= LOGE) ? 1 : (L <= 2 * LOGE ? 2 : 3);
+    constexpr int A1 = L < LOGE ? L : LOGE;
+    constexpr int A2 = (L - LOGE) < LOGE ? (L - LOGE) : LOGE;
+    constexpr int A3 = L - 2 * LOGE;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(st + (size_t)(tl * 8 + (c ^ (tl & 7))) * 8);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[c * 4 + q] = __half22float2(h2[q]);
+    }
+    stages<A1>(v);
+    if constexpr (NR >= 2) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            *reinterpret_cast<float4*>(rowbuf + swz(tl * E + 2 * i)) = make_float4(v[i].x, v[i].y, v[i + 1].x, v[i + 1].y);
+        named_bar(bar_id, T);
+        rload<LOGE, A2>(v, rowbuf, tl, T);
+        stages<A2>(v);
+    }
+    if constexpr (NR >= 3) {
+        rstore<LOGE, LOGE>(v, rowbuf, tl, T);
+        named_bar(bar_id, T);
+        rload<2 * LOGE, A3>(v, rowbuf, tl, T);
+        stages<A3>(v);
+    }
+}
+
+// Writes v (in the last round's layout) to the row buffer in natural order,
+// swizzled: element i at rowbuf[swz(i)].
+template <int L>
+__device__ __forceinline__ void store_natural(const float2 (&v)[32], float* rowbuf, int tl, int T) {
+    constexpr int NR = (L <= LOGE) ? 1 : (L <= 2 * LOGE ? 2 : 3);
+    constexpr int A2 = (L - LOGE) < LOGE ? (L - LOGE) : LOGE;
+    constexpr int A3 = L - 2 * LOGE;
+    if constexpr (NR == 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            *reinterpret_cast<float4*>(rowbuf + swz(tl * E + 2 * i)) = make_float4(v[i].x, v[i].y, v[i + 1].x, v[i + 1].y);
+    } else if constexpr (NR == 2) {
+        rstore<LOGE, A2>(v, rowbuf, tl, T);
+    } else {
+        rstore<2 * LOGE, A3>(v, rowbuf, tl, T);
+    }
+}
+
+template <int L, int MAXT>
+__global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
     const int K = p.K;
     const int T = K / E;
     const int R = blockDim.x / T;
     const int team = threadIdx.x / T;
     const int t = threadIdx.x % T;
+    const int lane = threadIdx.x & 31;
+    float* rowbufs = reinterpret_cast<float*>(smem_raw);
+    float* rowbuf = rowbufs + (size_t)team * K;
+    __half* stages0 = reinterpret_cast<__half*>(rowbufs + (size_t)R * K);
+    __half* stage0 = stages0 + (size_t)team * 2 * K;
+    uint32_t* gsm = reinterpret_cast<uint32_t*>(stages0 + (size_t)R * 2 * K);   // [256] group max bits, then s
+    float* red = reinterpret_cast<float*>(gsm + 256) + team * 16;
+    float* s_sm = reinterpret_cast<float*>(gsm);
     const int bar_id = 1 + team;
-    __shared__ float red[8][16];
+    const int stride = gridDim.x * R;
+    const int r0 = blockIdx.x * R + team;
 
-    float d = 1.0f;
-    if (!p.unit_scales) {
-        const float sg = p.s[(t * E) / p.G];
-        d = (sg == 0.0f) ? 1.0f : sg;
-    } else if (p.s_unit_out && blockIdx.x == 0) {
-        for (int g = threadIdx.x; g < K / p.G; g += blockDim.x) p.s_unit_out[g] = 1.0f;
+    auto issue_row = [&](int r, int sb) {
+        const __half* src = p.X + (size_t)r * K;
+        __half* dst = stage0 + (size_t)sb * K;
+        for (int u = t; u < K / 8; u += T) {
+            const int owner = u >> 3;
+            const int c = u & 7;
+            cp_async16(dst + (size_t)(owner * 8 + (c ^ (owner & 7))) * 8, src + (size_t)u * 8);
+        }
+    };
+
+    for (int g = threadIdx.x; g < 256; g += blockDim.x) gsm[g] = 0u;
+
+    if (p.phase & 1) {
+        // ------------------------------------------------------------- phase A
+        float2 m[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m[i] = make_float2(0.0f, 0.0f);
+        int it = 0;
+        if (r0 < p.rows) issue_row(r0, 0);
+        cp_async_commit();
+        for (int r = r0; r < p.rows; r += stride, ++it) {
+            const int sb = it & 1;
+            if (r + stride < p.rows) issue_row(r + stride, sb ^ 1);
+            cp_async_commit();
+            cp_async_wait<1>();
+            named_bar(bar_id, T);
+            const int tl = opaque(t);
+            float2 v[32];
+            rotate_row<L>(v, rowbuf, stage0 + (size_t)sb * K, tl, T, bar_id);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                m[i].x = fmaxf(m[i].x, fabsf(v[i].x));
+                m[i].y = fmaxf(m[i].y, fabsf(v[i].y));
+            }
+            named_bar(bar_id, T);   // row buffer and staging free for the next row
+        }
+        cp_async_wait<0>();
+        // the channel maxima of this team, in natural order, then over the teams
+        store_natural<L>(m, rowbuf, opaque(t), T);
+        __syncthreads();
+        if (R > 1) {
+            for (int i = threadIdx.x; i < K; i += blockDim.x) {
+                float mx = rowbufs[swz(i)];
+                for (int q = 1; q < R; ++q) mx = fmaxf(mx, rowbufs[(size_t)q * K + swz(i)]);
+                rowbufs[swz(i)] = mx;
+            }
+            __syncthreads();
+        }
+        // group maxima through the reorder index: a warp covers 32 consecutive
+        // positions j, all in one group (G is a multiple of 128)
+        for (int j = threadIdx.x; j < K; j += blockDim.x) {
+            float mx = rowbufs[swz(__ldg(p.perm + j))];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0 && mx > 0.0f) atomicMax(&gsm[j / p.G], __float_as_uint(mx));
+        }
+        __syncthreads();
+        for (int g = threadIdx.x; g < p.NG; g += blockDim.x)
+            p.partial[(size_t)blockIdx.x * p.NG + g] = __fmul_rn(p.c_n, __uint_as_float(gsm[g]));
+        if (!grid_barrier(p.gbar, p.err, p.limit_ns)) return;
+        for (int g = threadIdx.x; g < p.NG; g += blockDim.x) {
+            float mx = 0.0f;
+            for (int b = 0; b < (int)gridDim.x; ++b) mx = fmaxf(mx, __ldcg(p.partial + (size_t)b * p.NG + g));
+            s_sm[g] = mx;
+            if (blockIdx.x == 0) p.s[g] = mx;
+        }
+    } else {
+        for (int g = threadIdx.x; g < p.NG; g += blockDim.x) {
+            const float v = p.unit_scales ? 1.0f : p.s[g];
+            s_sm[g] = v;
+            if (p.unit_scales && blockIdx.x == 0) p.s[g] = 1.0f;
+        }
     }
+    if (!(p.phase & 2)) return;
+    __syncthreads();
+
+    // --------------------------------------------------------------- phase B
+    int it = 0;
+    if (r0 < p.rows) issue_row(r0, 0);
+    cp_async_commit();
+    // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
+    // perm is staged through shared memory: coalesced 16-byte global loads, and
+    // 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
+    // chunk reads below are bank-conflict free.
+    uint32_t gaddr[32];
+    {
+        int4* pst = reinterpret_cast<int4*>(rowbufs);
+        const int4* pg = reinterpret_cast<const int4*>(p.perm);
+        for (int c = threadIdx.x; c < K / 4; c += blockDim.x) pst[c ^ ((c >> 4) & 7)] = pg[c];
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int c = t * 16 + q;
+            const int4 v = pst[c ^ ((c >> 4) & 7)];
+            gaddr[2 * q] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
+            gaddr[2 * q + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
+        }
+        __syncthreads();   // the row buffers reuse this space
+    }
+    float d = s_sm[(t * E) / p.G];
+    if (d == 0.0f) d = 1.0f;
     const float yd = __frcp_rn(d);
     const float2 nd2 = make_float2(-d, -d), yd2 = make_float2(yd, yd);
+    const float2 c2 = make_float2(p.c_n, p.c_n);
     constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer, half to even
     const float2 magic2 = make_float2(kMagic, kMagic);
+    const bool divide = !p.unit_scales;
 
-    const int stride = gridDim.x * R;
-    for (int r = blockIdx.x * R + team; r < p.rows; r += stride) {
-        const float4* src = reinterpret_cast<const float4*>(p.xp + (size_t)r * K);
+    for (int r = r0; r < p.rows; r += stride, ++it) {
+        const int sb = it & 1;
+        if (r + stride < p.rows) issue_row(r + stride, sb ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        named_bar(bar_id, T);
+        const int tl = opaque(t);
+        float2 v[32];
+        rotate_row<L>(v, rowbuf, stage0 + (size_t)sb * K, tl, T, bar_id);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], c2);   // X_rot = c_n * v
+        store_natural<L>(v, rowbuf, tl, T);
+        named_bar(bar_id, T);
+
+        // gather X'[j] = X_rot[perm[j]], smooth, per-thread max
         float2 x[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 f = __ldcs(src + i * T + t);
-            x[2 * i] = make_float2(f.x, f.y);
-            x[2 * i + 1] = make_float2(f.z, f.w);
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t g0 = gaddr[2 * q], g1 = gaddr[2 * q + 1];
+            x[2 * q] = make_float2(rowbuf[g0 & 0xFFFFu], rowbuf[g0 >> 16]);
+            x[2 * q + 1] = make_float2(rowbuf[g1 & 0xFFFFu], rowbuf[g1 >> 16]);
         }
         float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            if (!p.unit_scales) x[i] = div_markstein(x[i], nd2, yd2);
+            if (divide) x[i] = div_markstein(x[i], nd2, yd2);
             amax = fmaxf(amax, fmaxf(fabsf(x[i].x), fabsf(x[i].y)));
         }
-        float tmx = amax;   // this thread's max |x~|
+        const float tmx = amax;   // this thread's max |x~|
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if ((t & 31) == 0) red[team][t >> 5] = amax;
-        named_bar(bar_id, T);
-        amax = red[team][0];
-        for (int w = 1; w < T / 32; ++w) amax = fmaxf(amax, red[team][w]);
+        if ((t & 31) == 0) red[t >> 5] = amax;
+        named_bar(bar_id, T);     // also: every thread of the team has gathered from the row buffer
+        amax = red[0];
+        for (int w = 1; w < T / 32; ++w) amax = fmaxf(amax, red[w]);
         const float scale = __fdiv_rn(amax, 7.0f);
 
         uint32_t pk[8], q8[16];
@@ -342,6 +438,7 @@ __global__ void __launch_bounds__(MAXT) smooth_quant_kernel(QuantArgs p) {
 #pragma unroll
             for (int w = 0; w < 8; ++w) {   // 8 elements (4 float2) per packed word
                 uint32_t b[8];
+                uint32_t e8[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     float2 z = div_markstein(x[4 * w + h], ns2, ys2);
@@ -352,25 +449,35 @@ __global__ void __launch_bounds__(MAXT) smooth_quant_kernel(QuantArgs p) {
                     z = __fadd2_rn(z, magic2);   // low bits: the rounded code, two's complement
                     b[2 * h] = __float_as_uint(z.x);
                     b[2 * h + 1] = __float_as_uint(z.y);
+                    if (p.a8_mode == 2) {
+                        const float2 cv = __fadd2_rn(z, make_float2(-kMagic, -kMagic));   // the code as an exact float
+                        e8[h] = e4m3x2(cv.x, cv.y);
+                    }
                 }
                 const uint32_t lo = low_bytes(b[0], b[2], b[4], b[6]);   // codes of k = 0, 2, 4, 6
                 const uint32_t hi = low_bytes(b[1], b[3], b[5], b[7]);   // codes of k = 1, 3, 5, 7
                 pk[w] = (lo & 0x0F0F0F0Fu) | ((hi << 4) & 0xF0F0F0F0u);
-                q8[2 * w] = lo;
-                q8[2 * w + 1] = hi;
+                if (p.a8_mode == 2) {
+                    q8[2 * w] = e8[0] | (e8[1] << 16);
+                    q8[2 * w + 1] = e8[2] | (e8[3] << 16);
+                } else {
+                    q8[2 * w] = lo;
+                    q8[2 * w + 1] = hi;
+                }
             }
         }
         uint4* dq = reinterpret_cast<uint4*>(p.qX + (size_t)r * (K / 2) + (size_t)t * 32);
         dq[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         dq[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        uint4* d8 = reinterpret_cast<uint4*>(p.qX8 + (size_t)r * K + (size_t)t * 64);
+        if (p.a8_mode) {
+            uint4* d8 = reinterpret_cast<uint4*>(p.a8 + (size_t)r * K + (size_t)t * 64);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d8[i] = make_uint4(q8[4 * i], q8[4 * i + 1], q8[4 * i + 2], q8[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) d8[i] = make_uint4(q8[4 * i], q8[4 * i + 1], q8[4 * i + 2], q8[4 * i + 3]);
+        }
         if (t == 0) p.scale_t[r] = scale;
-        named_bar(bar_id, T);   // red[] reused by the next row
     }
+    cp_async_wait<0>();
 }
-
 // Packed INT4 rows -> int8 GEMM operand rows (same k order as smooth_quant_kernel).
 __global__ void expand_kernel(const uint8_t* qX, int8_t* qX8, size_t nwords) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwords; i += (size_t)gridDim.x * blockDim.x) {
@@ -383,13 +490,29 @@ __global__ void expand_kernel(const uint8_t* qX, int8_t* qX8, size_t nwords) {
     }
 }
 
-// Packed INT4 weight rows -> int8 operand rows holding 16 q (the nibble in
-// the high half of each byte), in the k order of expand_kernel.  The GEMM's
-// epilogue expects the factor 16 on the weight side.
-__global__ void expand_weights_kernel(const uint8_t* qW, int8_t* qW8, size_t nwords) {
+// Packed INT4 rows -> e4m3 codes in natural k order (byte 2i from the low
+// nibble of packed byte i, byte 2i + 1 from its high nibble).  A nibble n is
+// the two's-complement code q = n - 16 * (n >> 3); its e4m3 byte comes from a
+// 16-entry table held in two pairs of registers and read with byte permutes.
+__device__ __forceinline__ uint32_t e4m3_of_nibbles(uint32_t nib4) {
+    // nib4: four nibbles, one per byte (values 0..15).  Codes 0..7 (n < 8) and
+    // -8..-1 (n >= 8) read separate 8-entry tables, selected per byte.
+    const uint32_t idx = nib4 & 0x07070707u;
+    const uint32_t sel = __byte_perm(idx | (idx >> 4), 0u, 0x0020) & 0x7777u;
+    // e4m3 of 0..7 and of -8..-1
+    const uint32_t pos = __byte_perm(0x44403800u, 0x4E4C4A48u, sel);
+    const uint32_t neg = __byte_perm(0xCACCCED0u, 0xB8C0C4C8u, sel);
+    const uint32_t negmask = ((nib4 >> 3) & 0x01010101u) * 0xFFu;
+    return (pos & ~negmask) | (neg & negmask);
+}
+
+__global__ void expand_e4m3_kernel(const uint8_t* q, uint8_t* out, size_t nwords) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwords; i += (size_t)gridDim.x * blockDim.x) {
-        const uint32_t w = reinterpret_cast<const uint32_t*>(qW)[i];
-        reinterpret_cast<uint2*>(qW8)[i] = make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
+        const uint32_t w = reinterpret_cast<const uint32_t*>(q)[i];
+        // bytes b0..b3 hold codes (2i, 2i+1): output order lo0 hi0 lo1 hi1 ...
+        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+        const uint32_t elo = e4m3_of_nibbles(lo), ehi = e4m3_of_nibbles(hi);
+        reinterpret_cast<uint2*>(out)[i] = make_uint2(__byte_perm(elo, ehi, 0x5140), __byte_perm(elo, ehi, 0x7362));
     }
 }
 
@@ -404,78 +527,87 @@ __global__ void divide_check_kernel(const float* a, const float* b, int n, float
     }
 }
 
+
+
 template <int L>
-static cudaError_t launch_rot(const RotArgs& a, int threads, int R, size_t smem, int nsm, cudaStream_t st) {
-    auto kern = threads <= CTA ? rot_gather_kernel<L, CTA> : rot_gather_kernel<L, 512>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+static cudaError_t launch_act(const ActArgs& a, int threads, size_t smem, int grid_cap, cudaStream_t st) {
+    auto kern = threads <= CTA ? act_kernel<L, CTA> : act_kernel<L, 512>;
+    static KernelSetup setup[2];
+    int occ = 0;
+    cudaError_t e = kernel_setup(reinterpret_cast<const void*>(kern), threads, smem, setup[threads <= CTA ? 0 : 1], &occ);
     if (e != cudaSuccess) return e;
+    const int nsm = device_sm_count();
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    const int R = threads / (a.K / E);
     int grid = (a.rows + R - 1) / R;
-    if (grid > nsm) grid = nsm;
-    kern<<<grid, threads, smem, st>>>(a);
-    return cudaGetLastError();
+    if (grid > occ * nsm) grid = occ * nsm;
+    if (grid > grid_cap) grid = grid_cap;
+    ActArgs args = a;
+    void* params[] = {&args};
+    // all CTAs must be resident together: the phases meet at a grid-wide barrier
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(threads), params, smem, st);
 }
 
 }  // namespace fast
 
 bool prep_fast_supported(int K, int n) {
-    return K % 2048 == 0 && K / 64 <= 512 && n >= 1 && n <= 8192;
+    // whole warps per row team, at most 512 threads, and the row buffers of a CTA in shared memory
+    return K % 2048 == 0 && K / 64 <= 512 && n >= 1 && n <= 8192 && fast::act_smem_bytes(K) <= 227 * 1024;
 }
 
-size_t prep_fast_scratch_bytes(int M, int K) { return (size_t)M * K * 4; }
+int prep_fast_rows_per_cta(int K) { return fast::act_rows_per_cta(K); }
 
 cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t st) {
     using namespace fast;
     const int K = pl.K;
     const int T = K / E;
-    int R = T <= CTA ? CTA / T : 1;
+    const int R = act_rows_per_cta(K);
     const int threads = T * R;
-    const size_t smem = (size_t)R * K * 4 + (size_t)R * 2 * K * 2;
+    const size_t smem = act_smem_bytes(K);
     int L = 0;
     while ((1 << L) < pl.n) ++L;
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-
+    ActArgs a;
+    a.X = reinterpret_cast<const __half*>(pl.X);
+    a.rows = pl.rows;
+    a.K = K;
+    a.G = pl.G;
+    a.NG = K / pl.G;
+    a.c_n = pl.c_n;
+    a.perm = pl.perm;
+    a.phase = pl.unit_scales ? 2 : pl.phase;
+    a.unit_scales = pl.unit_scales;
+    a.s = pl.s;
+    a.qX = pl.qX;
+    a.a8 = reinterpret_cast<uint8_t*>(pl.qX8);
+    a.a8_mode = pl.qX8 == nullptr ? 0 : (pl.a_e4m3 ? 2 : 1);
+    a.scale_t = pl.scale_t;
+    a.partial = pl.partial;
+    a.gbar = pl.gbar;
+    a.err = pl.err;
+    a.limit_ns = kWaitLimitNs;
     cudaError_t e;
-    if (!pl.unit_scales) {
-        e = cudaMemsetAsync(pl.s, 0, sizeof(float) * (size_t)(K / pl.G), st);
-        if (e != cudaSuccess) return e;
-    }
-    RotArgs ra;
-    ra.X = reinterpret_cast<const __half*>(pl.X);
-    ra.rows = pl.rows;
-    ra.K = K;
-    ra.G = pl.G;
-    ra.c_n = pl.c_n;
-    ra.perm = pl.perm;
-    ra.xp = pl.scratch;
-    ra.smax = pl.unit_scales ? nullptr : reinterpret_cast<uint32_t*>(pl.s);
     switch (L) {
-#define RRS_ROT_CASE(LL) \
-    case LL: e = launch_rot<LL>(ra, threads, R, smem, nsm, st); break;
-        RRS_ROT_CASE(0) RRS_ROT_CASE(1) RRS_ROT_CASE(2) RRS_ROT_CASE(3) RRS_ROT_CASE(4)
-        RRS_ROT_CASE(5) RRS_ROT_CASE(6) RRS_ROT_CASE(7) RRS_ROT_CASE(8) RRS_ROT_CASE(9)
-        RRS_ROT_CASE(10) RRS_ROT_CASE(11) RRS_ROT_CASE(12) RRS_ROT_CASE(13)
-#undef RRS_ROT_CASE
+#define RRS_ACT_CASE(LL) \
+    case LL: e = launch_act<LL>(a, threads, smem, pl.partial_rows, st); break;
+        RRS_ACT_CASE(0) RRS_ACT_CASE(1) RRS_ACT_CASE(2) RRS_ACT_CASE(3) RRS_ACT_CASE(4)
+        RRS_ACT_CASE(5) RRS_ACT_CASE(6) RRS_ACT_CASE(7) RRS_ACT_CASE(8) RRS_ACT_CASE(9)
+        RRS_ACT_CASE(10) RRS_ACT_CASE(11) RRS_ACT_CASE(12) RRS_ACT_CASE(13)
+#undef RRS_ACT_CASE
         default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess) return e;
+    return e;
+}
 
-    QuantArgs qa;
-    qa.xp = pl.scratch;
-    qa.rows = pl.rows;
-    qa.K = K;
-    qa.G = pl.G;
-    qa.unit_scales = pl.unit_scales;
-    qa.s = pl.s;
-    qa.qX = pl.qX;
-    qa.qX8 = pl.qX8;
-    qa.scale_t = pl.scale_t;
-    qa.s_unit_out = pl.unit_scales ? pl.s : nullptr;
-    int grid = (pl.rows + R - 1) / R;
-    if (grid > 4 * nsm) grid = 4 * nsm;
-    if (threads <= CTA) smooth_quant_kernel<CTA><<<grid, threads, 0, st>>>(qa);
-    else smooth_quant_kernel<512><<<grid, threads, 0, st>>>(qa);
+namespace fast {
+__global__ void fill_kernel(float* p, int n, float v) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
+}
+}  // namespace fast
+
+cudaError_t launch_fill(float* p, int n, float v, cudaStream_t st) {
+    int blocks = (n + 255) / 256;
+    if (blocks > 1024) blocks = 1024;
+    fast::fill_kernel<<<blocks, 256, 0, st>>>(p, n, v);
     return cudaGetLastError();
 }
 
@@ -490,24 +622,21 @@ cudaError_t launch_divide_check(const float* a, const float* b, int n, float* q_
 
 cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStream_t st) {
     const size_t nwords = (size_t)M * K / 8;
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = device_sm_count();
     size_t blocks = (nwords + 255) / 256;
     if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
     fast::expand_kernel<<<(unsigned)blocks, 256, 0, st>>>(qX, qX8, nwords);
     return cudaGetLastError();
 }
 
-cudaError_t launch_expand_weights(const uint8_t* qW, int8_t* qW8, int N, int K, cudaStream_t st) {
-    const size_t nwords = (size_t)N * K / 8;
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+cudaError_t launch_expand_e4m3(const uint8_t* q, uint8_t* out, int rows, int K, cudaStream_t st) {
+    const size_t nwords = (size_t)rows * K / 8;
+    const int nsm = device_sm_count();
     size_t blocks = (nwords + 255) / 256;
     if (blocks > (size_t)nsm * 8) blocks = (size_t)nsm * 8;
-    fast::expand_weights_kernel<<<(unsigned)blocks, 256, 0, st>>>(qW, qW8, nwords);
+    fast::expand_e4m3_kernel<<<(unsigned)blocks, 256, 0, st>>>(q, out, nwords);
     return cudaGetLastError();
 }
+
 
 }  // namespace rrs

@@ -124,6 +124,35 @@ rrs_status rrs_smooth_quant(const void *X, int M, int K, int G, int had_block, c
                             uint8_t *qX, float *s, float *scale_t, void *ws, size_t ws_bytes,
                             unsigned flags, rrs_stream_t stream);
 
+/* The two passes of rrs_smooth_quant as separate calls, for one batch whose
+ * tokens are split across devices (or calls).  The runtime scale of a group is
+ * the maximum over ALL tokens of the batch (summary page, "Approach": the
+ * smoothing scales are computed at inference from the activations), and a
+ * maximum of maxima is exact, so
+ *     rrs_group_max on every shard -> elementwise MAX of the shards' s (for
+ *     example an all-reduce with the MAX operation) -> rrs_smooth_quant_scaled
+ *     on every shard with that s
+ * gives, row for row, the same qX and scale_t bits (and the same s) as one
+ * rrs_smooth_quant over the whole batch.
+ *
+ * rrs_group_max (pass A): s[g] = max over this call's M tokens and the channels
+ * of group g of |X'|, fp32 [K/G] (0 for a group that is zero on every token).
+ * Under RRS_FORCE_UNIT_SCALES it writes s = 1.  Same arguments, limits,
+ * workspace (rrs_workspace_size(M, 0, K, G, had_block, flags) bytes) and errors
+ * as rrs_smooth_quant. */
+rrs_status rrs_group_max(const void *X, int M, int K, int G, int had_block, const int32_t *perm, float *s,
+                         void *ws, size_t ws_bytes, unsigned flags, rrs_stream_t stream);
+
+/* rrs_smooth_quant_scaled (pass B): qX and scale_t of this call's M tokens,
+ * each group divided by the given s[g] (a zero s[g] divides by 1), exactly as
+ * rrs_smooth_quant's second pass does.  s is an input, fp32 [K/G] device.
+ * RRS_FORCE_UNIT_SCALES is refused (RRS_ERR_INVALID_ARG): pass s filled with 1.
+ * With RRS_W_EXPANDED it also leaves the fp8 GEMM operand in the workspace,
+ * like rrs_smooth_quant.  Otherwise as rrs_smooth_quant. */
+rrs_status rrs_smooth_quant_scaled(const void *X, int M, int K, int G, int had_block, const int32_t *perm,
+                                   const float *s, uint8_t *qX, float *scale_t, void *ws, size_t ws_bytes,
+                                   unsigned flags, rrs_stream_t stream);
+
 /* Group-scaled W4A4 GEMM (rebuttal page "Novelty": the smoothing scale is
  * applied group-wise to match the hardware GEMM): exact int32 P_g per group
  * on the tensor cores, Y = (sum_g s_g * P_g) * scale_t * scale_w in fp32.

@@ -45,7 +45,12 @@ def test_library_is_sm100a_build():
 
 
 def test_workspace_size(L):
-    assert L.rrs_workspace_size(2048, 4096, 4096, 128, 4096, 0) >= 256
+    # header + the GEMM operand (M*K bytes) + one row of K/128 group maxima per CTA of
+    # the activation kernel; nothing of size M*K*4 (the rotation is recomputed, not stored)
+    need = L.rrs_workspace_size(2048, 4096, 4096, 128, 4096, 0)
+    assert 256 + 2048 * 4096 <= need < 256 + 2048 * 4096 + 2048 * 4096 // 4
+    # decode sizes keep room for the split-k partial sums of the GEMM
+    assert L.rrs_workspace_size(16, 8192, 8192, 128, 8192, 0) >= 256 + 16 * 8192 + 16 * 16 * 8192 * 4
 
 
 def test_perm_from_channel_max_host(L):
@@ -85,8 +90,21 @@ def test_argument_checks_fail_before_any_launch(L):
     # workspace too small
     assert L.rrs_smooth_quant(ok, 16, 256, 128, 256, ok, ok, ok, ok, ws, 8, 0, None) == 5
     need = L.rrs_workspace_size(16, 16, 4096, 128, 4096, 0)
-    assert need >= 256 + 16 * 4096 + 16 * 4096 * 4
-    assert L.rrs_smooth_quant(ok, 16, 4096, 128, 4096, ok, ok, ok, ok, ws, need - 1, 0, None) == 5
+    assert need >= 256 + 16 * 4096 + 16 * 16 * 16 * 4      # header, operand, split-k room
+    need_sq = L.rrs_workspace_size(16, 0, 4096, 128, 4096, 0)     # N = 0: no GEMM split-k room
+    assert 256 + 16 * 4096 <= need_sq <= need
+    assert L.rrs_smooth_quant(ok, 16, 4096, 128, 4096, ok, ok, ok, ok, ws, need_sq - 1, 0, None) == 5
+    # pass A / pass B of the token-sharded path: same checks
+    assert L.rrs_group_max(None, 16, 256, 128, 256, ok, ok, ws, 1 << 20, 0, None) == 1
+    assert L.rrs_group_max(ok, 0, 256, 128, 256, ok, ok, ws, 1 << 20, 0, None) == 1
+    assert L.rrs_group_max(ok, 16, 256, 64, 256, ok, ok, ws, 1 << 20, 0, None) == 2
+    assert L.rrs_group_max(ok, 16, 4096, 128, 4096, ok, ok, ws, need_sq - 1, 0, None) == 5
+    assert L.rrs_smooth_quant_scaled(ok, 16, 256, 128, 256, ok, None, ok, ok, ws, 1 << 20, 0, None) == 1
+    assert L.rrs_smooth_quant_scaled(ok, 16, 256, 100, 256, ok, ok, ok, ok, ws, 1 << 20, 0, None) == 1
+    assert L.rrs_smooth_quant_scaled(ok, 16, 4096, 128, 4096, ok, ok, ok, ok, ws, need_sq - 1, 0, None) == 5
+    # the scales come from s: unit scales do not apply to pass B
+    assert L.rrs_smooth_quant_scaled(ok, 16, 256, 128, 256, ok, ok, ok, ok, ws, 1 << 20, 2, None) == 1
+    assert b"s filled with 1" in L.rrs_last_error_string()
     # M < 1
     assert L.rrs_w4a4_gemm(ok, ok, ok, ok, ok, 0, 16, 256, 128, ok, ws, 1 << 20, 0, None) == 1
     assert L.rrs_debug_wait_timeout(0, ws, 256, None) == 1
@@ -126,7 +144,7 @@ def test_binding_flag_and_dtype_inference_without_gpu():
     assert b._y_flags(torch.empty(2, 2, dtype=torch.bfloat16), 0) == b.Y_BF16
     assert b._y_dtype(b.Y_BF16 | b.W_EXPANDED) == torch.bfloat16
     assert b._y_dtype(b.W_EXPANDED) == torch.float32
-    # packed weights are uint8 [N, K/2]; expanded ones int8 [N, K]; host tensors are refused
+    # packed weights are uint8 [N, K/2]; expanded ones e4m3 [N, K]; host tensors are refused
     with pytest.raises(TypeError):
         b._need_weights(torch.zeros(4, 64, dtype=torch.int8), 4, 128, 0)
     with pytest.raises(TypeError):
@@ -134,7 +152,7 @@ def test_binding_flag_and_dtype_inference_without_gpu():
     with pytest.raises(ValueError):
         b._need_weights(torch.zeros(4, 64, dtype=torch.uint8), 4, 128, 0)
     with pytest.raises(ValueError):
-        b._need_weights(torch.zeros(4, 128, dtype=torch.int8), 4, 128, b.W_EXPANDED)
+        b._need_weights(torch.zeros(4, 128, dtype=torch.float8_e4m3fn), 4, 128, b.W_EXPANDED)
 
 
 def test_next_row_bindings_refuse_host_tensors():

@@ -36,6 +36,11 @@ def assert_bits_equal(gpu, orc, what):
     assert bad[0].size == 0, f"{what}: {bad[0].size} mismatches, first at {[b[0] for b in bad]}"
 
 
+def min_workspace(M, K):
+    """The smallest workspace rrs_w4a4_gemm accepts: header + int8 operand, no room to split k."""
+    return torch.zeros(256 + (M * K + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
+
+
 def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
     """Runs the CUDA path and the oracle on the same inputs and compares."""
     K = X.shape[1]
@@ -46,13 +51,15 @@ def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
     qX, s, st = rrs.smooth_quant(Xd, pd, G, n, flags)
     ws = rrs.make_workspace(X.shape[0], W.shape[0], K, G, n, flags)
     Y = rrs.w4a4_gemm(qX, s, st, qW, sw, G, ws=ws)
-    # the expanded-weight kernel computes the same exact partials and the same
-    # fp32 promotion in the same order: its Y must be bit-identical
+    # the expanded-weight (fp8) kernel computes the same exact partials and the same
+    # fp32 promotion in the same order as the packed kernel when that one does not
+    # split k (a workspace with no room for partial sums): its Y must be bit-identical
     qW8 = rrs.expand_weights(qW)
     Y8 = rrs.w4a4_gemm(qX, s, st, qW8, sw, G, ws=ws, flags=rrs.W_EXPANDED)
+    Y1 = rrs.w4a4_gemm(qX, s, st, qW, sw, G, ws=min_workspace(X.shape[0], K))
     rrs.check_workspace(ws)
     torch.cuda.synchronize()
-    assert_bits_equal(Y8, Y, "Y (expanded weights) vs Y (packed weights)")
+    assert_bits_equal(Y8, Y1, "Y (expanded weights) vs Y (packed weights, unsplit)")
 
     _, oqX, os_, ost = oracle.smooth_quant(X, G, n_eff, perm.numpy(), unit_scales=unit)
     assert_bits_equal(s, os_, "s")
@@ -63,11 +70,12 @@ def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
     assert_bits_equal(qW, oqW, "qW")
     if check_y:
         Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
-        Yg = Y.cpu().numpy() if rows is None else Y.cpu().numpy()[rows]
-        ok = oracle.y_tolerance_ok(Yg, Yo, B)
-        assert ok.all(), f"Y: {np.count_nonzero(~ok)} of {ok.size} outside tolerance"
-        rel = np.linalg.norm(Yg - Yo) / max(np.linalg.norm(Yo), 1e-30)
-        assert rel < 1e-5
+        for Yt, what in ((Y, "Y"), (Y8, "Y (expanded weights)")):
+            Yg = Yt.cpu().numpy() if rows is None else Yt.cpu().numpy()[rows]
+            ok = oracle.y_tolerance_ok(Yg, Yo, B)
+            assert ok.all(), f"{what}: {np.count_nonzero(~ok)} of {ok.size} outside tolerance"
+            rel = np.linalg.norm(Yg - Yo) / max(np.linalg.norm(Yo), 1e-30)
+            assert rel < 1e-5
     return dict(qX=qX, s=s, st=st, qW=qW, sw=sw, Y=Y)
 
 
@@ -96,13 +104,24 @@ def test_tiny_partials_bit_exact(rrs):
     assert_bits_equal(P, oracle.group_partials(oqX, oqW, L.G), "P_g")
 
 
+# e4m3 bytes of the codes -8..7: sign, 4 exponent bits (bias 7), 3 mantissa bits
+# (OCP FP8 e4m3 format), written out by hand from the format's definition.
+E4M3_OF_CODE = {-8: 0xD0, -7: 0xCE, -6: 0xCC, -5: 0xCA, -4: 0xC8, -3: 0xC4, -2: 0xC0, -1: 0xB8,
+                0: 0x00, 1: 0x38, 2: 0x40, 3: 0x44, 4: 0x48, 5: 0x4A, 6: 0x4C, 7: 0x4E}
+
+
 def expanded_operand(q_packed: np.ndarray) -> np.ndarray:
-    """16 q per byte, k order 0,2,4,6,1,3,5,7 within each 8 codes (from the oracle's packed codes)."""
+    """The codes one per byte as e4m3, natural k order (from the oracle's packed codes)."""
     N, K2 = q_packed.shape
     codes = oracle.unpack(q_packed, 2 * K2).astype(np.int32)          # [N, K] natural k order
-    order = np.array([0, 2, 4, 6, 1, 3, 5, 7])
-    idx = (np.arange(2 * K2).reshape(-1, 8)[:, order]).reshape(-1)
-    return (16 * codes[:, idx]).astype(np.int8)
+    lut = np.array([E4M3_OF_CODE[c] for c in range(-8, 8)], dtype=np.uint8)
+    return lut[codes + 8]
+
+
+def test_e4m3_table_decodes_to_the_codes():
+    """The hand-written e4m3 table decodes (by torch's fp8 type) to the integer codes."""
+    b = torch.tensor([E4M3_OF_CODE[c] for c in range(-8, 8)], dtype=torch.uint8)
+    assert b.view(torch.float8_e4m3fn).float().tolist() == [float(c) for c in range(-8, 8)]
 
 
 def test_expand_weights_operand_bit_exact(rrs):
@@ -111,7 +130,11 @@ def test_expand_weights_operand_bit_exact(rrs):
     perm = wl.random_perm(L.K, 3)
     _, oqW, _ = oracle.prepare_weights(W, L.had_block, perm.numpy())
     qW8 = rrs.expand_weights(torch.from_numpy(oqW).to(DEV))
-    assert_bits_equal(qW8, expanded_operand(oqW), "qW8")
+    assert_bits_equal(qW8.view(torch.uint8), expanded_operand(oqW), "qW8")
+    # every code pattern: all 256 packed bytes in one row
+    allb = np.tile(np.arange(256, dtype=np.uint8), (4, 1))
+    assert_bits_equal(rrs.expand_weights(torch.from_numpy(allb).to(DEV)).view(torch.uint8),
+                      expanded_operand(allb), "qW8 (all byte values)")
 
 
 @pytest.mark.parametrize("M,N,K,G", [(130, 520, 1024, 128), (257, 136, 512, 256)])
@@ -122,6 +145,43 @@ def test_partials_bit_exact_expanded_weights(rrs, M, N, K, G):
     qW8 = rrs.expand_weights(torch.from_numpy(qW).to(DEV))
     P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(qX).to(DEV), qW8, G, flags=rrs.W_EXPANDED)
     assert_bits_equal(P, oracle.group_partials(qX, qW, G), "P_g (expanded weights)")
+
+
+# Shapes with at least 74 tiles of 256 x 256 take the CTA-pair kernel of the fp8
+# GEMM; ragged M and N (not multiples of 256) exercise its edge tiles.
+PAIR_SHAPES = [(300, 19016, 384, 128), (512, 18944, 512, 256), (260, 20480, 256, 256)]
+
+
+@pytest.mark.parametrize("M,N,K,G", PAIR_SHAPES)
+def test_pair_tiles_partials_bit_exact(rrs, M, N, K, G):
+    rng = np.random.default_rng(M * 3 + N)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    qW8 = rrs.expand_weights(torch.from_numpy(qW).to(DEV))
+    P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(qX).to(DEV), qW8, G, flags=rrs.W_EXPANDED)
+    assert_bits_equal(P, oracle.group_partials(qX, qW, G), "P_g (CTA-pair tiles)")
+
+
+@pytest.mark.parametrize("M,N,K,G", PAIR_SHAPES)
+def test_pair_tiles_y_matches_oracle_and_packed_kernel(rrs, M, N, K, G):
+    rng = np.random.default_rng(M + 7 * N)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    s = (rng.random(K // G, dtype=np.float32) + 0.5).astype(np.float32)
+    st = rng.random(M, dtype=np.float32)
+    sw = rng.random(N, dtype=np.float32)
+    qXd, sd, std, qWd, swd = (torch.from_numpy(a).to(DEV) for a in (qX, s, st, qW, sw))
+    Y8 = rrs.w4a4_gemm(qXd, sd, std, rrs.expand_weights(qWd), swd, G, flags=rrs.W_EXPANDED)
+    Y = rrs.w4a4_gemm(qXd, sd, std, qWd, swd, G)
+    Yb = rrs.w4a4_gemm(qXd, sd, std, rrs.expand_weights(qWd), swd, G, flags=rrs.W_EXPANDED,
+                       Y=torch.empty((M, N), dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert_bits_equal(Y8, Y, "Y (CTA-pair fp8 tiles) vs Y (packed kernel)")
+    assert torch.equal(Yb, Y8.to(torch.bfloat16)), "bf16 Y is the fp32 Y rounded"
+    rows = np.unique(np.concatenate([np.arange(4), np.arange(M - 4, M), rng.integers(0, M, 8)]))
+    Yo, B = oracle.linear_rows(qX, s, st, qW, sw, G, rows=rows)
+    ok = oracle.y_tolerance_ok(Y8.cpu().numpy()[rows], Yo, B)
+    assert ok.all(), f"{np.count_nonzero(~ok)} outside tolerance"
 
 
 @pytest.mark.parametrize("M,N", [(130, 520), (67, 200)])
@@ -184,12 +244,15 @@ def test_split_k_group_sizes_and_expanded_weights(rrs, M, N, K, G):
     qXd, sd, std, qWd, swd = (torch.from_numpy(a).to(DEV) for a in (qX, s, st, qW, sw))
     ws = rrs.make_workspace(M, N, K, G, 1)
     Y = rrs.w4a4_gemm(qXd, sd, std, qWd, swd, G, ws=ws)
+    Y1 = rrs.w4a4_gemm(qXd, sd, std, qWd, swd, G, ws=min_workspace(M, K))   # no split
     Y8 = rrs.w4a4_gemm(qXd, sd, std, rrs.expand_weights(qWd), swd, G, ws=ws, flags=rrs.W_EXPANDED)
     torch.cuda.synchronize()
-    assert_bits_equal(Y8, Y, "Y (expanded, split) vs Y (packed, split)")
+    # the fp8 kernel does not split k: same promotion order as the unsplit packed kernel
+    assert_bits_equal(Y8, Y1, "Y (expanded) vs Y (packed, unsplit)")
     Yo, B = oracle.linear_rows(qX, s, st, qW, sw, G)
-    ok = oracle.y_tolerance_ok(Y.cpu().numpy(), Yo, B)
-    assert ok.all(), f"{np.count_nonzero(~ok)} outside tolerance"
+    for Yg in (Y, Y8):
+        ok = oracle.y_tolerance_ok(Yg.cpu().numpy(), Yo, B)
+        assert ok.all(), f"{np.count_nonzero(~ok)} outside tolerance"
 
 
 @pytest.mark.parametrize("M,K,G,n,flags", [(1, 2048, 128, 2048, 0), (3, 4096, 256, 4096, 0), (16, 8192, 128, 8192, 0),
