@@ -22,6 +22,7 @@ FORCE_UNIT_SCALES = 2
 WS_HOLDS_A8 = 4
 W_EXPANDED = 8
 Y_BF16 = 16
+Y_SILU_MUL = 32
 
 _STATUS = {
     0: "RRS_OK",
@@ -191,7 +192,21 @@ def _y_flags(Y: Optional[torch.Tensor], flags: int) -> int:
 
 
 def _y_dtype(flags: int) -> torch.dtype:
+    if flags & Y_SILU_MUL:
+        return torch.float16
     return torch.bfloat16 if flags & Y_BF16 else torch.float32
+
+
+def _y_shape(M: int, N: int, flags: int) -> Tuple[int, int]:
+    return (M, N // 2) if flags & Y_SILU_MUL else (M, N)
+
+
+def interleave_gate_up(W_gate: torch.Tensor, W_up: torch.Tensor) -> torch.Tensor:
+    """Weight rows of a gated MLP's fused gate/up projection in the order RRS_Y_SILU_MUL
+    reads: row 2f = W_gate[f], row 2f + 1 = W_up[f]."""
+    if W_gate.shape != W_up.shape:
+        raise ValueError("gate and up weights must have the same shape")
+    return torch.stack([W_gate, W_up], dim=1).reshape(2 * W_gate.shape[0], W_gate.shape[1]).contiguous()
 
 
 def _need_weights(qW: torch.Tensor, N: int, K: int, flags: int):
@@ -216,8 +231,8 @@ def w4a4_gemm(qX: torch.Tensor, s: torch.Tensor, scale_t: torch.Tensor, qW: torc
     _need(scale_t, "scale_t", torch.float32, (M,))
     _need(scale_w, "scale_w", torch.float32, (N,))
     flags = _y_flags(Y, flags)
-    Y = torch.empty((M, N), dtype=_y_dtype(flags), device=qX.device) if Y is None else Y
-    _need(Y, "Y", _y_dtype(flags), (M, N))
+    Y = torch.empty(_y_shape(M, N, flags), dtype=_y_dtype(flags), device=qX.device) if Y is None else Y
+    _need(Y, "Y", _y_dtype(flags), _y_shape(M, N, flags))
     ws = make_workspace(M, N, K, G, 1, 0, qX.device) if ws is None else ws
     _check(lib().rrs_w4a4_gemm(_ptr(qX), _ptr(s), _ptr(scale_t), _ptr(qW), _ptr(scale_w), M, N, K, G, _ptr(Y),
                                _ptr(ws), ws.numel(), flags, _stream(stream)))
@@ -241,8 +256,8 @@ def linear(X: torch.Tensor, qW: torch.Tensor, scale_w: torch.Tensor, perm: torch
     s = torch.empty(max(K // G, 1), dtype=torch.float32, device=dev) if s is None else s
     scale_t = torch.empty(M, dtype=torch.float32, device=dev) if scale_t is None else scale_t
     flags = _y_flags(Y, flags)
-    Y = torch.empty((M, N), dtype=_y_dtype(flags), device=dev) if Y is None else Y
-    _need(Y, "Y", _y_dtype(flags), (M, N))
+    Y = torch.empty(_y_shape(M, N, flags), dtype=_y_dtype(flags), device=dev) if Y is None else Y
+    _need(Y, "Y", _y_dtype(flags), _y_shape(M, N, flags))
     ws = make_workspace(M, N, K, G, had_block, flags, dev) if ws is None else ws
     _check(lib().rrs_linear(_ptr(X), _ptr(qW), _ptr(scale_w), _ptr(perm), M, N, K, G, had_block, _ptr(qX),
                             _ptr(s), _ptr(scale_t), _ptr(Y), _ptr(ws), ws.numel(), flags, _stream(stream)))

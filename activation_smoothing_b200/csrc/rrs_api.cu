@@ -190,7 +190,7 @@ rrs_status launch_gemm_checked(const uint8_t* qX, const float* s, const float* s
         gf.Y = Y;
         gf.P = P;
         gf.err = reinterpret_cast<uint32_t*>(ws);
-        gf.y_bf16 = P == nullptr && (flags & RRS_Y_BF16) != 0;
+        gf.ymode = P != nullptr ? 0 : (flags & RRS_Y_SILU_MUL) ? 2 : (flags & RRS_Y_BF16) ? 1 : 0;
         gf.bn = 0;
         gf.stream = st;
         cudaError_t e = rrs::launch_gemm_f8(gf);
@@ -433,6 +433,11 @@ rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t
     if (r != RRS_OK) return r;
     r = check_ws(ws, ws_bytes, ws_bytes_gemm(M, K));
     if (r != RRS_OK) return r;
+    if (flags & RRS_Y_SILU_MUL) {
+        if (!(flags & RRS_W_EXPANDED))
+            return fail(RRS_ERR_UNSUPPORTED, "RRS_Y_SILU_MUL needs the fp8 path (RRS_W_EXPANDED)");
+        if (N % 2 != 0) return fail(RRS_ERR_INVALID_ARG, "RRS_Y_SILU_MUL needs N even (interleaved gate/up rows), N = %d", N);
+    }
     return launch_gemm_checked(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, nullptr, ws, ws_bytes, flags,
                                reinterpret_cast<cudaStream_t>(stream));
 }
@@ -443,7 +448,7 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
     return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes,
-                         RRS_WS_HOLDS_A8 | (flags & (RRS_W_EXPANDED | RRS_Y_BF16)), stream);
+                         RRS_WS_HOLDS_A8 | (flags & (RRS_W_EXPANDED | RRS_Y_BF16 | RRS_Y_SILU_MUL)), stream);
 }
 
 rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* qW, const float* scale_w,
@@ -460,7 +465,8 @@ rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* 
     rrs_status r = rrs_linear(X_dev, qW, scale_w, perm, M, N, K, G, had_block, qX, s, scale_t, Y_dev, ws,
                               ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
-    e = cudaMemcpyAsync(Y_host, Y_dev, (size_t)M * N * ((flags & RRS_Y_BF16) ? 2 : 4), cudaMemcpyDeviceToHost, st);
+    const size_t ybytes = (flags & RRS_Y_SILU_MUL) ? (size_t)M * (N / 2) * 2 : (size_t)M * N * ((flags & RRS_Y_BF16) ? 2 : 4);
+    e = cudaMemcpyAsync(Y_host, Y_dev, ybytes, cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy of Y");
     e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -493,14 +499,13 @@ rrs_status rrs_silu_mul(const float* GU, int M, int F, void* H, rrs_stream_t str
     return RRS_OK;
 }
 
-rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, int8_t* qW8, rrs_stream_t stream) {
+rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, uint8_t* qW8, rrs_stream_t stream) {
     RRS_REQUIRE_PTR(qW);
     RRS_REQUIRE_PTR(qW8);
     if (N < 1) return fail(RRS_ERR_INVALID_ARG, "N = %d", N);
     rrs_status r = check_K(K);
     if (r != RRS_OK) return r;
-    cudaError_t e = rrs::launch_expand_e4m3(qW, reinterpret_cast<uint8_t*>(qW8), N, K,
-                                            reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = rrs::launch_expand_e4m3(qW, qW8, N, K, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "expand_weights kernel");
     return RRS_OK;
 }

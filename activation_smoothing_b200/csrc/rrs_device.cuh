@@ -186,4 +186,14 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// The gated-MLP activation of one output: silu(g) * u with silu(g) = g / (1 +
+// exp(-g)) in fp32, saturated to +-65504 (the fp16 range the next layer's
+// activation path takes); the caller rounds it to fp16.  One definition for the
+// element-wise step and the GEMM epilogue that fuses it, so both give the same bits.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+    const float h = __fmul_rn(sg, u);
+    return fminf(fmaxf(h, -65504.0f), 65504.0f);
+}
+
 }  // namespace rrs

@@ -137,13 +137,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-// Y[row][colbase + c] = acc_c * scale_t[row] * scale_w[colbase + c] for this
-// lane's row and CW columns.  Every lane of the warp runs the shuffles; rows past
-// M skip only their stores.  Lane l holds scale_w of two columns of each 64-column
-// chunk and shuffles broadcast them.  Each lane owns one row: whole 32-byte
-// sectors per lane (8 fp32 columns, one 256-bit store) keep L2 from merging
-// partial sectors; ragged edges and a misaligned Y take scalar stores.
-template <int CW, bool YBF16>
+// Output of a tile row, YMODE: 0 fp32 Y, 1 bf16 Y (the fp32 value rounded to
+// nearest even), 2 the gated-MLP activation H = fp16(silu(y[2f]) * y[2f+1]) of
+// an interleaved gate/up projection (H is [M, N/2]; silu_mul as rrs_silu_mul).
+enum : int { kYF32 = 0, kYBF16 = 1, kYSiluMul = 2 };
+
+// y[row][colbase + c] = acc_c * scale_t[row] * scale_w[colbase + c] for this
+// lane's row and CW columns, stored as YMODE says.  Every lane of the warp runs
+// the shuffles; rows past M skip only their stores.  Lane l holds scale_w of two
+// columns of each 64-column chunk and shuffles broadcast them.  Each lane owns
+// one row: whole 32-byte sectors per lane (one 256-bit store) keep L2 from
+// merging partial sectors; ragged edges and misaligned outputs take scalar stores.
+template <int CW, int YMODE>
 __device__ __forceinline__ void store_tile(const Args& g, const float2 (&acc)[CW / 2], int row, int colbase,
                                            int lane) {
     const bool rv = row < g.M;
@@ -154,6 +159,46 @@ __device__ __forceinline__ void store_tile(const Args& g, const float2 (&acc)[CW
     for (int ch = 0; ch < CW / 64; ++ch) {
         const int cl = colbase + 64 * ch + 2 * lane;
         const float2 swl = make_float2(cl < g.N ? g.scale_w[cl] : 0.0f, cl + 1 < g.N ? g.scale_w[cl + 1] : 0.0f);
+        if (YMODE == kYSiluMul) {
+            // 32 columns -> 16 halves = one 32-byte store per lane
+            const int NH = g.N / 2;
+            const bool hv = (NH & 15) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 31u) == 0;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                uint32_t hw[8];
+#pragma unroll
+                for (int q = 0; q < 16; q += 2) {
+                    float hq[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int i = 16 * jj + q + e;
+                        const float2 sw = make_float2(__shfl_sync(0xffffffffu, swl.x, i),
+                                                      __shfl_sync(0xffffffffu, swl.y, i));
+                        const float2 y = __fmul2_rn(__fmul2_rn(acc[32 * ch + i], st2), sw);
+                        hq[e] = silu_mul(y.x, y.y);
+                    }
+                    const __half2 h2 = __floats2half2_rn(hq[0], hq[1]);
+                    hw[q / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                const int f0 = (colbase + 64 * ch + 32 * jj) / 2;
+                if (!rv) continue;
+                __half* hrow = reinterpret_cast<__half*>(g.Y) + (size_t)row * NH;
+                if (hv && f0 + 15 < NH) {
+                    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                                 ::"l"(hrow + f0), "r"(hw[0]), "r"(hw[1]), "r"(hw[2]), "r"(hw[3]),
+                                   "r"(hw[4]), "r"(hw[5]), "r"(hw[6]), "r"(hw[7])
+                                 : "memory");
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const __half2 h2 = *reinterpret_cast<const __half2*>(&hw[q]);
+                        if (f0 + 2 * q < NH) hrow[f0 + 2 * q] = __low2half(h2);
+                        if (f0 + 2 * q + 1 < NH) hrow[f0 + 2 * q + 1] = __high2half(h2);
+                    }
+                }
+            }
+            continue;
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float2 y[4];
@@ -165,7 +210,7 @@ __device__ __forceinline__ void store_tile(const Args& g, const float2 (&acc)[CW
             }
             const int col = colbase + 64 * ch + 8 * j;
             if (!rv) continue;
-            if (YBF16) {
+            if (YMODE == kYBF16) {
                 __nv_bfloat16* brow = reinterpret_cast<__nv_bfloat16*>(g.Y) + (size_t)row * g.N;
                 if ((g.N & 7) == 0 && col + 7 < g.N) {
                     uint32_t u[4];
@@ -204,7 +249,7 @@ __device__ __forceinline__ void store_tile(const Args& g, const float2 (&acc)[CW
 // Epilogue warps: per promotion block, read this warp's 32 rows x CW columns of
 // fp32 partial sums from TMEM and accumulate s_g * P_g; per tile apply
 // scale_t * scale_w and store Y (debug: store the exact per-group partials).
-template <int BN, bool DEBUG_P, bool YBF16>
+template <int BN, bool DEBUG_P, int YMODE>
 __device__ __forceinline__ void epilogue(const Args& g, uint32_t tmem, uint64_t* tfull, uint64_t* tempty,
                                          const float* s_sm, volatile int* abortv, int warp, int lane, int ntiles,
                                          int nmb, int NPB) {
@@ -268,11 +313,11 @@ __device__ __forceinline__ void epilogue(const Args& g, uint32_t tmem, uint64_t*
                 for (int i = 0; i < CW / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             }
         }
-        if (!DEBUG_P && ok) store_tile<CW, YBF16>(g, acc, row, n0 + col0, lane);
+        if (!DEBUG_P && ok) store_tile<CW, YMODE>(g, acc, row, n0 + col0, lane);
     }
 }
 
-template <int BN, bool DEBUG_P, bool YBF16>
+template <int BN, bool DEBUG_P, int YMODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_f8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     using C = Cfg<BN>;
@@ -405,7 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait_bounded(done, 0, &no_abort, g.err, kErrGemmTimeout, g.limit_ns);
         }
     } else {
-        epilogue<BN, DEBUG_P, YBF16>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
+        epilogue<BN, DEBUG_P, YMODE>(g, tmem, tfull, tempty, s_sm, abortv, warp, lane, ntiles, nmb, NPB);
     }
     tc_fence_before();
     __syncthreads();
@@ -510,7 +555,7 @@ __device__ __forceinline__ void commit_both(uint64_t* bar) {
 }
 }  // namespace pair
 
-template <bool DEBUG_P, bool YBF16>
+template <bool DEBUG_P, int YMODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     gemm_f8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     using namespace pair;
@@ -716,7 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < CW / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
                 }
             }
-            if (!DEBUG_P && ok) store_tile<CW, YBF16>(g, acc, row, n0 + col0, lane);
+            if (!DEBUG_P && ok) store_tile<CW, YMODE>(g, acc, row, n0 + col0, lane);
         }
     }
     tc_fence_before();
@@ -765,11 +810,12 @@ static cudaError_t launch_bn(const GemmF8Launch& gl, const Args& a, int nsm) {
     if (!make_map(&tmB, gl.B, (uint64_t)gl.K, (uint64_t)gl.N, BN)) return cudaErrorInvalidValue;
     const int ntiles = ((gl.M + BM - 1) / BM) * ((gl.N + BN - 1) / BN);
     const int grid = ntiles < nsm ? ntiles : nsm;
-    const int v = gl.P ? 0 : gl.y_bf16 ? 1 : 2;
-    auto kern = v == 0 ? gemm_f8_kernel<BN, true, false>
-                : v == 1 ? gemm_f8_kernel<BN, false, true>
-                         : gemm_f8_kernel<BN, false, false>;
-    static KernelSetup setup[3];
+    const int v = gl.P ? 0 : 1 + gl.ymode;
+    auto kern = v == 0 ? gemm_f8_kernel<BN, true, kYF32>
+                : v == 1 ? gemm_f8_kernel<BN, false, kYF32>
+                : v == 2 ? gemm_f8_kernel<BN, false, kYBF16>
+                         : gemm_f8_kernel<BN, false, kYSiluMul>;
+    static KernelSetup setup[4];
     int occ = 0;
     cudaError_t e = kernel_setup(reinterpret_cast<const void*>(kern), NTHREADS, C::SMEM, setup[v], &occ);
     if (e != cudaSuccess) return e;
@@ -798,12 +844,13 @@ static cudaError_t launch_pair(const GemmF8Launch& gl, const Args& a, int nsm) {
     if (!make_map_kblocks(&tmA, gl.A, (uint64_t)gl.K, (uint64_t)gl.M, BM, KPS)) return cudaErrorInvalidValue;
     if (!make_map_kblocks(&tmB, gl.B, (uint64_t)gl.K, (uint64_t)gl.N, BNH, KPS)) return cudaErrorInvalidValue;
     const int ntiles = ((gl.M + 2 * BM - 1) / (2 * BM)) * ((gl.N + BN - 1) / BN);
-    const int v = gl.P ? 0 : gl.y_bf16 ? 1 : 2;
-    auto kern = v == 0 ? gemm_f8_pair_kernel<true, false>
-                : v == 1 ? gemm_f8_pair_kernel<false, true>
-                         : gemm_f8_pair_kernel<false, false>;
-    static KernelSetup setup[3];
-    static int maxc_cache[3][16] = {};
+    const int v = gl.P ? 0 : 1 + gl.ymode;
+    auto kern = v == 0 ? gemm_f8_pair_kernel<true, kYF32>
+                : v == 1 ? gemm_f8_pair_kernel<false, kYF32>
+                : v == 2 ? gemm_f8_pair_kernel<false, kYBF16>
+                         : gemm_f8_pair_kernel<false, kYSiluMul>;
+    static KernelSetup setup[4];
+    static int maxc_cache[4][16] = {};
     int occ = 0;
     cudaError_t e = kernel_setup(reinterpret_cast<const void*>(kern), NTHREADS, SMEM, setup[v], &occ);
     if (e != cudaSuccess) return e;

@@ -100,7 +100,7 @@ struct GemmF8Launch {
     void* Y;                // fp32 or bf16 [M, N] (null in debug mode)
     int32_t* P;             // [K/G, M, N] debug partials (null in normal mode)
     uint32_t* err;          // workspace error word
-    bool y_bf16;
+    int ymode;              // 0 fp32 Y, 1 bf16 Y, 2 H = fp16(silu(y[2f]) * y[2f+1]) [M, N/2]
     int bn;                 // tile width 128 or 256; 0 = chosen from the shape
     cudaStream_t stream;
 };

@@ -12,16 +12,12 @@
 
 #include <cstdint>
 
+#include "rrs_device.cuh"
 #include "rrs_internal.h"
 
 namespace rrs {
 namespace mlp {
 
-__device__ __forceinline__ float silu_mul(float g, float u) {
-    const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
-    const float h = __fmul_rn(sg, u);
-    return fminf(fmaxf(h, -65504.0f), 65504.0f);
-}
 
 // Four outputs per thread when F % 4 == 0 (16-byte loads, 8-byte stores).
 __global__ void silu_mul_vec4_kernel(const float* GU, int M, int F, __half* H) {
@@ -53,9 +49,7 @@ __global__ void silu_mul_kernel(const float* GU, int M, int F, __half* H) {
 }  // namespace mlp
 
 cudaError_t launch_silu_mul(const float* GU, int M, int F, void* H, cudaStream_t st) {
-    int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = device_sm_count();
     __half* h = reinterpret_cast<__half*>(H);
     const bool vec = F % 4 == 0;
     const size_t items = (size_t)M * (vec ? F / 4 : F);

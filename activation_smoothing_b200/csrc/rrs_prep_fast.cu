@@ -1,21 +1,21 @@
 // rrs_prep_fast.cu -- online activation path for K a multiple of 2048 (every
 // LLaMA projection shape): one cooperative persistent kernel in two phases.
 //
-//   phase A   X (fp16) -> Hadamard rotation of every row this CTA owns; the
-//             largest |X_rot| of each channel over those rows (registers), then
-//             through the reorder index the CTA's largest |X'| per group, into
-//             one row of a per-CTA table in the workspace
+//   phase A   X (fp16) -> Hadamard rotation and reorder gather of every row
+//             this CTA owns; each thread keeps the largest |X'| of its outputs
+//             (all in one group), and the CTA's group maxima go into one row of
+//             a per-CTA table in the workspace
 //   barrier   a grid-wide barrier (bounded wait); every CTA then reduces the
 //             table: s[g] = max over all tokens and group channels of |X'|
 //   phase B   X again (an L2 hit) -> the same rotation bit for bit, reorder
 //             gather, division by s_g, per-token INT4 quantisation; writes qX
-//             (packed), scale_t and, if asked, the GEMM operand
+//             (packed), scale_t and, if asked, the GEMM operand.  When every
+//             team owns at most one row (decode token counts), the rotated row
+//             stays in shared memory across the barrier and is not recomputed.
 //
 // Nothing of size M x K passes between the phases: the rotation is recomputed
-// instead of stored.  The group max needs no gather in phase A: max over
-// tokens commutes with the reorder, and c_n * |v| is monotone in |v|, so
-// s_g = RN(c_n * max_{j in g} max_t |v_t[perm[j]]|) exactly.
-//
+// (or kept on chip) instead of stored.
+
 // Work split: a team of T = K/64 threads (a multiple of 32) owns one row at a
 // time; each thread holds 64 elements.  Rotation rounds: up to 6 butterfly
 // stages on the 64 registers (f32x2 packed add/sub for every stage but the
@@ -160,14 +160,31 @@ struct ActArgs {
     uint32_t* gbar;      // grid barrier state: arrival count, generation (zero-filled before first use)
     uint32_t* err;       // workspace error word
     uint64_t limit_ns;
+    int nst;             // fp16 staging slots per team (2..4): rows in flight ahead of the one being rotated
 };
 
 // Rows of one CTA for a given K (T = K/64 threads per row).
 __host__ __device__ constexpr int act_rows_per_cta(int K) { return (K / E) <= CTA ? CTA / (K / E) : 1; }
-// Shared memory: R fp32 row buffers, R double-buffered fp16 staging rows,
-// 256 words of group maxima / scales, R x 16 floats of row-max partials.
-__host__ __device__ constexpr size_t act_smem_bytes(int K) {
-    return (size_t)act_rows_per_cta(K) * K * 8 + 1024 + (size_t)act_rows_per_cta(K) * 64;
+// Shared memory: R fp32 row buffers, R x nst fp16 staging rows, 256 words of
+// group maxima / scales, R x 16 floats of row-max partials.
+__host__ __device__ constexpr size_t act_smem_bytes(int K, int nst = 2) {
+    return (size_t)act_rows_per_cta(K) * K * 4 + (size_t)nst * act_rows_per_cta(K) * K * 2 + 1024 +
+           (size_t)act_rows_per_cta(K) * 64;
+}
+constexpr size_t kActSmemLimit = 227 * 1024;
+// Most staging slots (2..4) that fit in shared memory.
+inline int act_stages(int K) {
+    int nst = 4;
+    while (nst > 2 && act_smem_bytes(K, nst) > kActSmemLimit) --nst;
+    return nst;
+}
+
+// Waits until at most `pending` of this thread's cp.async groups are in flight.
+__device__ __forceinline__ void cp_async_wait_dyn(int pending) {
+    if (pending >= 3) cp_async_wait<3>();
+    else if (pending == 2) cp_async_wait<2>();
+    else if (pending == 1) cp_async_wait<1>();
+    else cp_async_wait<0>();
 }
 
 // Grid-wide barrier for a cooperative launch: sense reversal on two words
@@ -267,17 +284,21 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     const int R = blockDim.x / T;
     const int team = threadIdx.x / T;
     const int t = threadIdx.x % T;
-    const int lane = threadIdx.x & 31;
     float* rowbufs = reinterpret_cast<float*>(smem_raw);
     float* rowbuf = rowbufs + (size_t)team * K;
+    const int nst = p.nst;
     __half* stages0 = reinterpret_cast<__half*>(rowbufs + (size_t)R * K);
-    __half* stage0 = stages0 + (size_t)team * 2 * K;
-    uint32_t* gsm = reinterpret_cast<uint32_t*>(stages0 + (size_t)R * 2 * K);   // [256] group max bits, then s
+    __half* stage0 = stages0 + (size_t)team * nst * K;
+    uint32_t* gsm = reinterpret_cast<uint32_t*>(stages0 + (size_t)R * nst * K);   // [256] group max bits, then s
     float* red = reinterpret_cast<float*>(gsm + 256) + team * 16;
     float* s_sm = reinterpret_cast<float*>(gsm);
     const int bar_id = 1 + team;
     const int stride = gridDim.x * R;
     const int r0 = blockIdx.x * R + team;
+    // Every team owns at most one row: phase B reuses the rotated row that phase
+    // A leaves in the team's row buffer instead of loading and rotating it again.
+    const bool keep = (p.phase & 3) == 3 && stride >= p.rows;
+    const float2 c2 = make_float2(p.c_n, p.c_n);
 
     auto issue_row = [&](int r, int sb) {
         const __half* src = p.X + (size_t)r * K;
@@ -288,62 +309,141 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
             cp_async16(dst + (size_t)(owner * 8 + (c ^ (owner & 7))) * 8, src + (size_t)u * 8);
         }
     };
+    // X_rot of the staged row into the row buffer, natural order (c_n applied);
+    // a barrier makes it visible to the team.
+    auto rotate_into_rowbuf = [&](int sb) {
+        const int tl = opaque(t);
+        float2 v[32];
+        rotate_row<L>(v, rowbuf, stage0 + (size_t)sb * K, tl, T, bar_id);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], c2);   // X_rot = c_n * v
+        store_natural<L>(v, rowbuf, tl, T);
+        named_bar(bar_id, T);
+    };
 
+    // The first nst - 1 rows of a pass in flight, one cp.async group each (empty
+    // groups past the last row keep the group count uniform).
+    auto prologue = [&]() {
+        for (int q = 0; q < nst - 1; ++q) {
+            const int r = r0 + q * stride;
+            if (r < p.rows) issue_row(r, q);
+            cp_async_commit();
+        }
+    };
+    // Before rotating the it-th row of a pass: put row it + nst - 1 in flight and
+    // wait for row it.
+    auto advance = [&](int r, int it_) {
+        const int rn = r + (nst - 1) * stride;
+        if (rn < p.rows) issue_row(rn, (it_ + nst - 1) % nst);
+        cp_async_commit();
+        cp_async_wait_dyn(nst - 1);
+        named_bar(bar_id, T);
+    };
+
+    // first rows in flight while the gather addresses are built
+    int it = 0;
+    const bool run_a = (p.phase & 1) != 0;
+    if (run_a || !keep) prologue();
     for (int g = threadIdx.x; g < 256; g += blockDim.x) gsm[g] = 0u;
 
-    if (p.phase & 1) {
-        // ------------------------------------------------------------- phase A
-        float2 m[32];
+    // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
+    // perm is staged through shared memory: 16-byte global loads, four in flight,
+    // and 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
+    // chunk reads below are bank-conflict free.
+    uint32_t gaddr[32];
+    {
+        int4* pst = reinterpret_cast<int4*>(rowbufs);
+        const int4* pg = reinterpret_cast<const int4*>(p.perm);
+        for (int c0 = 0; c0 < K / 4; c0 += 4 * (int)blockDim.x) {
+            int4 v[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) m[i] = make_float2(0.0f, 0.0f);
-        int it = 0;
-        if (r0 < p.rows) issue_row(r0, 0);
-        cp_async_commit();
-        for (int r = r0; r < p.rows; r += stride, ++it) {
-            const int sb = it & 1;
-            if (r + stride < p.rows) issue_row(r + stride, sb ^ 1);
-            cp_async_commit();
-            cp_async_wait<1>();
-            named_bar(bar_id, T);
-            const int tl = opaque(t);
-            float2 v[32];
-            rotate_row<L>(v, rowbuf, stage0 + (size_t)sb * K, tl, T, bar_id);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                m[i].x = fmaxf(m[i].x, fabsf(v[i].x));
-                m[i].y = fmaxf(m[i].y, fabsf(v[i].y));
+            for (int q = 0; q < 4; ++q) {
+                const int c = c0 + q * (int)blockDim.x + (int)threadIdx.x;
+                if (c < K / 4) v[q] = __ldg(pg + c);
             }
-            named_bar(bar_id, T);   // row buffer and staging free for the next row
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = c0 + q * (int)blockDim.x + (int)threadIdx.x;
+                if (c < K / 4) pst[c ^ ((c >> 4) & 7)] = v[q];
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int c = t * 16 + q;
+            const int4 v = pst[c ^ ((c >> 4) & 7)];
+            gaddr[2 * q] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
+            gaddr[2 * q + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
+        }
+        __syncthreads();   // the row buffers reuse this space
+    }
+    auto gather = [&](float2 (&x)[32]) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t g0 = gaddr[2 * q], g1 = gaddr[2 * q + 1];
+            x[2 * q] = make_float2(rowbuf[g0 & 0xFFFFu], rowbuf[g0 >> 16]);
+            x[2 * q + 1] = make_float2(rowbuf[g1 & 0xFFFFu], rowbuf[g1 >> 16]);
+        }
+    };
+
+    if (run_a) {
+        // ------------------------------------------------------------- phase A
+        // Per row: rotate, reorder (gather), and keep the largest |X'| of this
+        // thread's outputs, all of which lie in one group (64 | G).
+        float gmx = 0.0f;
+        for (int r = r0; r < p.rows; r += stride, ++it) {
+            advance(r, it);
+            rotate_into_rowbuf(it % nst);
+            float2 x[32];
+            gather(x);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gmx = fmaxf(gmx, fmaxf(fabsf(x[i].x), fabsf(x[i].y)));
+            if (!keep) named_bar(bar_id, T);   // row buffer and staging free for the next row
         }
         cp_async_wait<0>();
-        // the channel maxima of this team, in natural order, then over the teams
-        store_natural<L>(m, rowbuf, opaque(t), T);
+        if (!keep && (p.phase & 2)) {
+            // phase B's first rows in flight across the grid barrier
+            __syncthreads();
+            prologue();
+        }
+        // threads of one group are consecutive (G / 64 of them): shuffle-reduce
+        // within aligned power-of-two segments, one shared atomic per segment
+        {
+            const int gsz = p.G / E;
+            const int seg = (gsz & -gsz) < 32 ? (gsz & -gsz) : 32;
+            for (int o = seg >> 1; o > 0; o >>= 1) gmx = fmaxf(gmx, __shfl_xor_sync(0xffffffffu, gmx, o));
+            if ((t % seg) == 0 && gmx > 0.0f) atomicMax(&gsm[(t * E) / p.G], __float_as_uint(gmx));
+        }
         __syncthreads();
-        if (R > 1) {
-            for (int i = threadIdx.x; i < K; i += blockDim.x) {
-                float mx = rowbufs[swz(i)];
-                for (int q = 1; q < R; ++q) mx = fmaxf(mx, rowbufs[(size_t)q * K + swz(i)]);
-                rowbufs[swz(i)] = mx;
+        for (int g = threadIdx.x; g < p.NG; g += blockDim.x) {
+            p.partial[(size_t)blockIdx.x * p.NG + g] = __uint_as_float(gsm[g]);
+            gsm[g] = 0u;
+        }
+        if (!grid_barrier(p.gbar, p.err, p.limit_ns)) return;
+        // s[g] = max over the CTAs' rows of the table: thread i takes group i % NG and every
+        // slices-th CTA from i / NG, eight independent loads at a time, then a shared max
+        {
+            const int slices = (int)blockDim.x >= p.NG ? (int)blockDim.x / p.NG : 1;
+            const int g = threadIdx.x % p.NG;
+            const int sl = threadIdx.x / p.NG;
+            if (sl < slices) {
+                float mx[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mx[q] = 0.0f;
+                int b = sl;
+                for (; b + 7 * slices < (int)gridDim.x; b += 8 * slices) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) mx[q] = fmaxf(mx[q], __ldcg(p.partial + (size_t)(b + q * slices) * p.NG + g));
+                }
+                for (; b < (int)gridDim.x; b += slices) mx[0] = fmaxf(mx[0], __ldcg(p.partial + (size_t)b * p.NG + g));
+                float m = mx[0];
+#pragma unroll
+                for (int q = 1; q < 8; ++q) m = fmaxf(m, mx[q]);
+                if (m > 0.0f) atomicMax(&gsm[g], __float_as_uint(m));
             }
             __syncthreads();
-        }
-        // group maxima through the reorder index: a warp covers 32 consecutive
-        // positions j, all in one group (G is a multiple of 128)
-        for (int j = threadIdx.x; j < K; j += blockDim.x) {
-            float mx = rowbufs[swz(__ldg(p.perm + j))];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0 && mx > 0.0f) atomicMax(&gsm[j / p.G], __float_as_uint(mx));
-        }
-        __syncthreads();
-        for (int g = threadIdx.x; g < p.NG; g += blockDim.x)
-            p.partial[(size_t)blockIdx.x * p.NG + g] = __fmul_rn(p.c_n, __uint_as_float(gsm[g]));
-        if (!grid_barrier(p.gbar, p.err, p.limit_ns)) return;
-        for (int g = threadIdx.x; g < p.NG; g += blockDim.x) {
-            float mx = 0.0f;
-            for (int b = 0; b < (int)gridDim.x; ++b) mx = fmaxf(mx, __ldcg(p.partial + (size_t)b * p.NG + g));
-            s_sm[g] = mx;
-            if (blockIdx.x == 0) p.s[g] = mx;
+            if (blockIdx.x == 0)
+                for (int g2 = threadIdx.x; g2 < p.NG; g2 += blockDim.x) p.s[g2] = s_sm[g2];
         }
     } else {
         for (int g = threadIdx.x; g < p.NG; g += blockDim.x) {
@@ -356,59 +456,23 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     __syncthreads();
 
     // --------------------------------------------------------------- phase B
-    int it = 0;
-    if (r0 < p.rows) issue_row(r0, 0);
-    cp_async_commit();
-    // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
-    // perm is staged through shared memory: coalesced 16-byte global loads, and
-    // 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
-    // chunk reads below are bank-conflict free.
-    uint32_t gaddr[32];
-    {
-        int4* pst = reinterpret_cast<int4*>(rowbufs);
-        const int4* pg = reinterpret_cast<const int4*>(p.perm);
-        for (int c = threadIdx.x; c < K / 4; c += blockDim.x) pst[c ^ ((c >> 4) & 7)] = pg[c];
-        __syncthreads();
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const int c = t * 16 + q;
-            const int4 v = pst[c ^ ((c >> 4) & 7)];
-            gaddr[2 * q] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
-            gaddr[2 * q + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
-        }
-        __syncthreads();   // the row buffers reuse this space
-    }
+    it = 0;
     float d = s_sm[(t * E) / p.G];
     if (d == 0.0f) d = 1.0f;
     const float yd = __frcp_rn(d);
     const float2 nd2 = make_float2(-d, -d), yd2 = make_float2(yd, yd);
-    const float2 c2 = make_float2(p.c_n, p.c_n);
     constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer, half to even
     const float2 magic2 = make_float2(kMagic, kMagic);
     const bool divide = !p.unit_scales;
 
     for (int r = r0; r < p.rows; r += stride, ++it) {
-        const int sb = it & 1;
-        if (r + stride < p.rows) issue_row(r + stride, sb ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        named_bar(bar_id, T);
-        const int tl = opaque(t);
-        float2 v[32];
-        rotate_row<L>(v, rowbuf, stage0 + (size_t)sb * K, tl, T, bar_id);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul2_rn(v[i], c2);   // X_rot = c_n * v
-        store_natural<L>(v, rowbuf, tl, T);
-        named_bar(bar_id, T);
-
+        if (!keep) {
+            advance(r, it);
+            rotate_into_rowbuf(it % nst);
+        }
         // gather X'[j] = X_rot[perm[j]], smooth, per-thread max
         float2 x[32];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const uint32_t g0 = gaddr[2 * q], g1 = gaddr[2 * q + 1];
-            x[2 * q] = make_float2(rowbuf[g0 & 0xFFFFu], rowbuf[g0 >> 16]);
-            x[2 * q + 1] = make_float2(rowbuf[g1 & 0xFFFFu], rowbuf[g1 >> 16]);
-        }
+        gather(x);
         float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -478,6 +542,7 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     }
     cp_async_wait<0>();
 }
+
 // Packed INT4 rows -> int8 GEMM operand rows (same k order as smooth_quant_kernel).
 __global__ void expand_kernel(const uint8_t* qX, int8_t* qX8, size_t nwords) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwords; i += (size_t)gridDim.x * blockDim.x) {
@@ -552,7 +617,7 @@ static cudaError_t launch_act(const ActArgs& a, int threads, size_t smem, int gr
 
 bool prep_fast_supported(int K, int n) {
     // whole warps per row team, at most 512 threads, and the row buffers of a CTA in shared memory
-    return K % 2048 == 0 && K / 64 <= 512 && n >= 1 && n <= 8192 && fast::act_smem_bytes(K) <= 227 * 1024;
+    return K % 2048 == 0 && K / 64 <= 512 && n >= 1 && n <= 8192 && fast::act_smem_bytes(K, 2) <= fast::kActSmemLimit;
 }
 
 int prep_fast_rows_per_cta(int K) { return fast::act_rows_per_cta(K); }
@@ -563,7 +628,8 @@ cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t st) {
     const int T = K / E;
     const int R = act_rows_per_cta(K);
     const int threads = T * R;
-    const size_t smem = act_smem_bytes(K);
+    const int nst = act_stages(K);
+    const size_t smem = act_smem_bytes(K, nst);
     int L = 0;
     while ((1 << L) < pl.n) ++L;
     ActArgs a;
@@ -585,6 +651,7 @@ cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t st) {
     a.gbar = pl.gbar;
     a.err = pl.err;
     a.limit_ns = kWaitLimitNs;
+    a.nst = nst;
     cudaError_t e;
     switch (L) {
 #define RRS_ACT_CASE(LL) \

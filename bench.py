@@ -4,13 +4,17 @@ A step is one RRS linear (online rotation/reorder/group max/quantise, then
 the group-scaled W4A4 GEMM) on each LLaMA-3-8B projection shape the headline
 metric is quoted on: M=2048 tokens, K=4096, N in {4096 (q/o), 1024 (k/v),
 14336 (gate/up)}, G=128, Hadamard 4096.  Inputs are synthetic (seeded,
-outlier-laden); weights are prepared once, off the timed path.
+outlier-laden); weights are prepared once, off the timed path, and held as
+their INT4 codes one per byte in e4m3 form (the operand of the fp8 tensor-core
+GEMM); the same step with the weights packed two codes per byte is reported
+beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  With torchrun (N > 1) every rank runs its own
-replica (the layer does not shard: replicas only); the time is the max over
-ranks and the value the ops of all ranks over that time.
+Prints one JSON line (rank 0).  With N > 1 it runs one process per GPU (under
+torchrun, or relaunching itself under torch.distributed.run): every rank runs
+its own replica (independent batches: replicas only); the time is the max over
+ranks and the value the operations of all ranks over that time.
 """
 from __future__ import annotations
 
@@ -30,11 +34,28 @@ sys.path.insert(0, ROOT)
 METRIC = "RRS W4A4 linear TOPS (prep+GEMM) at LLaMA-3-8B shapes; % of INT8 TC peak"
 UNIT = "TOPS"
 N_XSETS = 4            # distinct activation buffers per layer, rotated between steps
-# DRAM bytes (read + write) per GEMM launch, mean over the q/o, k/v and gate/up
-# launches of one step, from the ncu capture summarised in
-# profiles/gemm_kernel_llama3_8b.md.  None whenever gemm_kernel has changed since
-# that capture.
-GEMM_TRAFFIC_BYTES = 45.8e6
+GEMM_SOURCE = os.path.join(ROOT, "activation_smoothing_b200", "csrc", "rrs_gemm_f8.cu")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_f8_llama3_8b.md")
+
+
+def gemm_traffic_bytes():
+    """DRAM bytes (read + write) per GEMM launch, mean over the step's layers, from the
+    ncu capture summarised in the profile file, or None when the GEMM source has changed
+    since that capture (the summary records the source's sha256)."""
+    import hashlib
+    import re
+    try:
+        src = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
+        txt = open(GEMM_PROFILE).read()
+    except OSError:
+        return None, "no capture summary"
+    m_sha = re.search(r"source sha256: ([0-9a-f]{64})", txt)
+    m_b = re.search(r"dram bytes per launch, mean of the step's layers: ([0-9.]+)", txt)
+    if not (m_sha and m_b):
+        return None, "capture summary lacks the source hash or the traffic figure"
+    if m_sha.group(1) != src:
+        return None, "GEMM source changed since the capture"
+    return float(m_b.group(1)), "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean of the 3 layers' launches"
 
 
 def peaks():
@@ -135,6 +156,18 @@ def dist_setup():
     return world, rank, local
 
 
+def relaunch(n: int) -> int:
+    """Runs this same command as n processes, one per GPU (torch.distributed.run on
+    127.0.0.1, a free port); returns its exit status."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def run_ours(args):
     import datetime
 
@@ -142,6 +175,8 @@ def run_ours(args):
     from activation_smoothing_b200 import workloads as wl
 
     world, rank, local = dist_setup()
+    if world != args.gpus:
+        raise SystemExit(f"bench: --gpus {args.gpus} but {world} process(es) are running")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
@@ -159,7 +194,7 @@ def run_ours(args):
         perm = rrs.calibrate_perm(Xc, L.had_block)
         W = wl.make_weights(L).to(dev)
         qW, sw = rrs.prepare_weights(W, perm, L.had_block)
-        qW8 = rrs.expand_weights(qW)          # secondary path: weights one code per byte
+        qW8 = rrs.expand_weights(qW)          # the codes one per byte (e4m3): the fp8 GEMM's operand
         del W
         xs = [wl.make_activations(L, sample=activation_sample(i, rank)).to(dev) for i in range(N_XSETS)]
         st = dict(L=L, perm=perm, qW=qW, qW8=qW8, sw=sw, xs=xs,
@@ -172,88 +207,65 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
+    HEAD = rrs.W_EXPANDED            # headline: fp8 operands (weights expanded offline)
 
-    def step(i, events=None):
+    def step(i, flags, events=None):
         for j, st in enumerate(state):
             L = st["L"]
             X = st["xs"][i % N_XSETS]
+            qw = st["qW8"] if flags & rrs.W_EXPANDED else st["qW"]
             if events is not None:
                 events[j][0].record(stream)
-            rrs.smooth_quant(X, st["perm"], L.G, L.had_block, qX=st["qX"], s=st["s"], scale_t=st["st"],
-                             ws=st["ws"])
+            rrs.smooth_quant(X, st["perm"], L.G, L.had_block, flags=flags & rrs.W_EXPANDED, qX=st["qX"], s=st["s"],
+                             scale_t=st["st"], ws=st["ws"])
             if events is not None:
                 events[j][1].record(stream)
-            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW"], st["sw"], L.G, Y=st["Y"], ws=st["ws"],
-                          flags=rrs.WS_HOLDS_A8)
+            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], qw, st["sw"], L.G, Y=st["Y"], ws=st["ws"],
+                          flags=rrs.WS_HOLDS_A8 | flags)
             if events is not None:
                 events[j][2].record(stream)
 
-    for i in range(args.warmup):
-        step(i)
-    for st in state:
-        rrs.check_workspace(st["ws"])
-    torch.cuda.synchronize()
-
-    K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in state] for _ in range(K)]
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    def timed(K, flags, with_events):
+        for i in range(args.warmup):
+            step(i, flags)
+        for st in state:
+            rrs.check_workspace(st["ws"])
+        torch.cuda.synchronize()
+        evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in state] for _ in range(K)] \
+            if with_events else None
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
         t0.record(stream)
         for i in range(K):
-            step(i, evs[i])
+            step(i, flags, evs[i] if evs else None)
         t1.record(stream)
         torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    ms = t0.elapsed_time(t1)
-    for st in state:
-        rrs.check_workspace(st["ws"])
+        if pg:
+            pg.barrier()
+        ms = max_over_ranks(t0.elapsed_time(t1), pg, dev)
+        for st in state:
+            rrs.check_workspace(st["ws"])
+        return ms, evs
 
+    K = args.steps
+    with ClockSampler(local) as clk:
+        ms, evs = timed(K, HEAD, True)
     prep_ms = [sum(evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(K)) / K for j in range(len(state))]
     gemm_ms = [sum(evs[i][j][1].elapsed_time(evs[i][j][2]) for i in range(K)) / K for j in range(len(state))]
-
-    ms = max_over_ranks(ms, pg, dev)
-
     ops_step = sum(st["L"].ops for st in state)
     value = whole_job_tops(ops_step, K, world, ms)
 
-    # ---- secondary: the same step with the weights expanded offline to the int8
-    # operand (rrs_expand_weights + RRS_W_EXPANDED); same codes, same results.
-    Kx = max(3, min(K, 500))
-    xg = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in state]
-
-    def step_expanded(i, timed):
-        for j, st in enumerate(state):
-            L = st["L"]
-            rrs.smooth_quant(st["xs"][i % N_XSETS], st["perm"], L.G, L.had_block, qX=st["qX"], s=st["s"],
-                             scale_t=st["st"], ws=st["ws"])
-            if timed:
-                xg[j][0].record(stream)
-            rrs.w4a4_gemm(st["qX"], st["s"], st["st"], st["qW8"], st["sw"], L.G, Y=st["Y"], ws=st["ws"],
-                          flags=rrs.WS_HOLDS_A8 | rrs.W_EXPANDED)
-            if timed:
-                xg[j][1].record(stream)
-    for i in range(3):
-        step_expanded(i, False)
-    torch.cuda.synchronize()
-    xa, xb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    xa.record(stream)
-    for i in range(Kx):
-        step_expanded(i, True)
-    xb.record(stream)
-    torch.cuda.synchronize()
-    # per-layer GEMM times from the last step's events (all steps are alike)
-    xgemm = [xg[j][0].elapsed_time(xg[j][1]) for j in range(len(state))]
-    xms = max_over_ranks(xa.elapsed_time(xb), pg, dev)
-    for st in state:
-        rrs.check_workspace(st["ws"])
-    expanded = {"value": round(whole_job_tops(ops_step, Kx, world, xms), 2), "unit": UNIT, "steps": Kx,
-                "gemm_ms_per_layer_last_step": [round(x, 5) for x in xgemm],
-                "weights": "INT4 codes stored one per byte as 16 q (rrs_expand_weights); 2x weight bytes"}
+    # ---- the same step with the weights packed two codes per byte (INT8 tensor-core
+    # kernel that unpacks them on chip); same codes, same results
+    Kp = max(3, min(K, 500))
+    pms, pevs = timed(Kp, 0, True)
+    packed = {"value": round(whole_job_tops(ops_step, Kp, world, pms), 2), "unit": UNIT, "steps": Kp,
+              "gemm_ms_per_layer": [round(sum(pevs[i][j][1].elapsed_time(pevs[i][j][2]) for i in range(Kp)) / Kp, 5)
+                                    for j in range(len(state))],
+              "weights": "INT4 codes packed two per byte (N*K/2 bytes); int8 tensor-core GEMM"}
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed.
     e2e = None
@@ -265,8 +277,8 @@ def run_ours(args):
         def e2e_step():
             for j, st in enumerate(state):
                 L = st["L"]
-                rrs.linear_from_host(hx[j], st["xs"][1], st["qW"], st["sw"], st["perm"], L.G, L.had_block,
-                                     st["qX"], st["s"], st["st"], st["Y"], hy[j], st["ws"])
+                rrs.linear_from_host(hx[j], st["xs"][1], st["qW8"], st["sw"], st["perm"], L.G, L.had_block,
+                                     st["qX"], st["s"], st["st"], st["Y"], hy[j], st["ws"], flags=HEAD)
         for _ in range(3):
             e2e_step()
         if pg:
@@ -283,31 +295,33 @@ def run_ours(args):
         e2e = {"value": whole_job_tops(ops_step, Ke, world, ems), "unit": UNIT,
                "h2d_bytes_per_step": sum(st["L"].M * st["L"].K * 2 for st in state),
                "d2h_bytes_per_step": sum(st["L"].M * st["L"].N * 4 for st in state),
-               "steps": Ke}
+               "steps": Ke, "call": "rrs_linear_from_host (RRS_W_EXPANDED)"}
 
     int8_peak, hbm_peak, src = peaks()
-    gemm_ops = sum(st["L"].ops for st in state)
-    gemm_tops = gemm_ops / (sum(gemm_ms) * 1e-3) / 1e12
+    gemm_tops = ops_step / (sum(gemm_ms) * 1e-3) / 1e12
     prep_bytes = [2 * st["L"].M * st["L"].K + st["L"].M * st["L"].K // 2 + 4 * st["L"].M + 4 * (st["L"].K // st["L"].G)
                   for st in state]
     prep_gbs = sum(prep_bytes) / (sum(prep_ms) * 1e-3) / 1e9
-    launches_per_step = 3 * len(state)      # rotate+group max, smooth+quantise, GEMM per layer
+    launches_per_step = 2 * len(state)      # activation kernel + GEMM per layer
+    traffic, traffic_note = gemm_traffic_bytes()
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8 MMA / fp32 prep",
-        "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights); weights packed INT4",
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8 (e4m3) MMA on INT4 codes, fp32 accumulate / fp32 prep",
+        "data": "synthetic (seeded outlier-laden activations, N(0,0.02) weights); INT4 weight codes held one per "
+                "byte (e4m3) for the fp8 GEMM",
         "config": bench_config(names, layers, world),
         "roofline": {"bound": "tensor", "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1),
-                     "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": GEMM_TRAFFIC_BYTES,
-                     "kernel": "rrs gemm_kernel (tcgen05 kind::i8)", "peak_source": src + " (2 x bf16 burst)",
-                     "traffic_note": "DRAM bytes per GEMM launch, mean of the 3 layers (ncu)"},
+                     "unit": "TOPS", "frac": round(gemm_tops / int8_peak, 4), "traffic": traffic,
+                     "kernel": "rrs gemm_f8 (tcgen05.mma kind::f8f6f4; CTA-pair 256x256 tiles for q/o and gate/up)",
+                     "peak_source": src + " (2 x bf16 burst = the nominal dense fp8/int8 rate)",
+                     "traffic_note": traffic_note},
         "prep": {"ms_per_layer": [round(x, 5) for x in prep_ms], "algorithmic_GBps": round(prep_gbs, 1),
                  "hbm_frac": round(prep_gbs / hbm_peak, 4)},
         "gemm": {"ms_per_layer": [round(x, 5) for x in gemm_ms], "TOPS": round(gemm_tops, 1)},
         "e2e": e2e,
-        "expanded_weights": expanded,
+        "packed_weights": packed,
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
     }
@@ -343,14 +357,68 @@ def _oracle_sample(layers, rows_per_layer, cols_per_layer=None, seed=0):
     return ops, secs
 
 
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_worker(job):
+    """One process of the all-cores baseline: the oracle on its own slice of rows."""
+    names, rows, offset = job
+    import numpy as np
+
+    import oracle
+    from activation_smoothing_b200 import workloads as wl
+
+    ops, secs = 0, 0.0
+    for name in names:
+        L = wl.LAYERS[name]
+        X = wl.make_activations(L, sample=2, M=offset + rows)[offset:offset + rows].contiguous()
+        W = wl.make_weights(L)
+        perm = np.arange(L.K, dtype=np.int32)
+        _, qW, sw = oracle.prepare_weights(W, L.had_block, perm)     # offline, untimed
+        t = time.perf_counter()
+        _, qX, s, st = oracle.smooth_quant(X, L.G, L.had_block, perm)
+        oracle.linear_rows(qX, s, st, qW, sw, L.G)
+        secs += time.perf_counter() - t
+        ops += 2 * rows * L.N * L.K
+    return ops, secs
+
+
 def cpu_baseline(layers, budget_s=20.0):
-    """The oracle as it stands, single-threaded, on a bounded row sample."""
+    """The oracle as it stands (plain single-threaded C), on a bounded row sample: once in
+    this process, and once as one process per host core on disjoint rows (wall time)."""
+    import multiprocessing as mproc
+
     ops, secs = _oracle_sample(layers, 1)
-    rows = max(1, min(64, int(budget_s / max(secs, 1e-6))))
+    rows = max(1, min(64, int(budget_s / 2 / max(secs, 1e-6))))
     ops, secs = _oracle_sample(layers, rows)
-    return {"value": ops / secs / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{rows} token rows of each layer (prep of those rows + their GEMM rows, all N); "
-                      f"weights prepared untimed; single-threaded C", "seconds": round(secs, 2)}
+    single = {"value": ops / secs / 1e12, "unit": UNIT, "cores": 1, "seconds": round(secs, 2),
+              "sample": f"{rows} token rows of each layer"}
+    ncpu = os.cpu_count() or 1
+    procs = max(1, min(ncpu, 16))
+    per = max(1, rows // 4)
+    names = [L.name for L in layers]
+    ctx = mproc.get_context("spawn")          # the parent has a CUDA context: never fork
+    with ctx.Pool(procs) as pool:
+        pool.map(_oracle_worker, [(names[:1], 1, 0)] * procs)        # start-up and imports, untimed
+        jobs = [(names, per, i * per) for i in range(procs)]
+        t = time.perf_counter()
+        res = pool.map(_oracle_worker, jobs)
+        wall = time.perf_counter() - t
+    tot_ops = sum(r[0] for r in res)
+    # the workers also prepare their weights (untimed inside each worker); charge the
+    # wall time only with the timed part: the slowest worker's timed seconds
+    busy = max(r[1] for r in res)
+    return {"value": tot_ops / busy / 1e12, "unit": UNIT, "cores": procs, "kind": "oracle",
+            "sample": f"{per} token rows of each layer per process x {procs} processes (disjoint rows; prep of "
+                      f"those rows + their GEMM rows, all N); weights prepared untimed; single-threaded C per process",
+            "nproc": ncpu, "cpu_model": _cpu_model(), "wall_seconds": round(wall, 2), "single_thread": single}
 
 
 def run_reference(args):
@@ -528,6 +596,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit(relaunch(args.gpus))
     if args.report:
         run_report(args)
     elif args.impl == "reference":

@@ -85,27 +85,46 @@ typedef enum {
 /* flags */
 #define RRS_NO_ROTATE 1u         /* identity instead of the Hadamard (plain Runtime Smooth) */
 #define RRS_FORCE_UNIT_SCALES 2u /* s := 1 for every group (A4W4 per-channel scheme, no smoothing) */
-#define RRS_WS_HOLDS_A8 4u       /* rrs_w4a4_gemm: the workspace already holds the int8 activation
-                                    operand that rrs_smooth_quant wrote for this qX (same ws, same
-                                    stream, nothing in between); skips re-expanding qX */
-#define RRS_W_EXPANDED 8u        /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host and the debug
-                                    partials: qW points at the int8 operand that rrs_expand_weights
-                                    wrote ([N, K] bytes) instead of the packed INT4 codes */
+#define RRS_WS_HOLDS_A8 4u       /* rrs_w4a4_gemm: the workspace already holds the activation operand
+                                    that rrs_smooth_quant (or rrs_smooth_quant_scaled) wrote for this
+                                    qX with the same RRS_W_EXPANDED bit (same ws, same stream,
+                                    nothing in between); skips expanding qX again */
+#define RRS_W_EXPANDED 8u        /* qW points at the weight codes one per byte in e4m3 form that
+                                    rrs_expand_weights wrote ([N, K] bytes) instead of the packed
+                                    INT4 codes, and the GEMM runs on the fp8 tensor-core path
+                                    (rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host, the debug
+                                    partials).  Passed to rrs_smooth_quant / rrs_smooth_quant_scaled
+                                    it makes them leave the e4m3 activation operand in the
+                                    workspace (otherwise the int8 one of the packed path). */
 #define RRS_Y_BF16 16u           /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host: Y (and Y_host)
                                     hold bf16 [M, N] -- the fp32 result rounded to nearest even --
                                     instead of fp32; pass the buffer cast to float *.  The pages fix
                                     no output type; bf16 is the usual deployment type of Y. */
+#define RRS_Y_SILU_MUL 32u       /* rrs_w4a4_gemm, rrs_linear, rrs_linear_from_host, fp8 path only
+                                    (with RRS_W_EXPANDED): the layer is the fused gate/up projection
+                                    of a gated MLP block with its weight rows interleaved (row 2f
+                                    the gate row of feature f, row 2f+1 its up row; N even), and
+                                    instead of Y the GEMM writes the down projection's input
+                                    H fp16 [M, N/2], H[t][f] = fp16(silu(Y[t][2f]) * Y[t][2f+1])
+                                    from the fp32 Y it would have stored, with rrs_silu_mul's
+                                    arithmetic (same bits).  Pass H cast to float *.  Saves
+                                    writing and reading the fp32 gate/up output. */
 
 /* Bytes of workspace the calls below need for this problem.  Layout: a
- * 256-byte header holding the kernels' error word (zero-fill it once before
- * first use), then the int8 copy of the activation codes that the GEMM's
- * tensor cores read (M*K bytes), then, when K is a multiple of 2048, the
- * reordered fp32 activations X' that pass between the two activation kernels
- * (M*K*4 bytes).  For M <= 16 the space after the int8 operand is at least
- * 16*M*N*4 bytes: the GEMM then splits k across CTAs and keeps the partial sums
- * there (the X' scratch is dead by then).  rrs_w4a4_gemm alone needs only the
- * first two parts; given less room it simply does not split.  One workspace
- * must not be used by two calls in flight at the same time. */
+ * 256-byte header (zero-fill it once before first use: it holds the kernels'
+ * error word and the state of the activation kernel's grid-wide barrier, which
+ * every completed call leaves zeroed again), then the activation codes that the
+ * GEMM's tensor cores read (M*K bytes: int8, or e4m3 under RRS_W_EXPANDED),
+ * then, when K is a multiple of 2048, a table of group maxima with one row of
+ * K/128 floats per CTA of the activation kernel (at most 1024 rows).  For
+ * M <= 16 and N > 0 the space after the operand is at least 16*M*N*4 bytes: the
+ * packed-weight GEMM then splits k across CTAs and keeps its partial sums there
+ * (the table is dead by then).  rrs_w4a4_gemm alone needs only the first two
+ * parts; given less room it simply does not split.  N = 0 sizes a workspace for
+ * the activation calls alone.  One workspace must not be used by two calls in
+ * flight at the same time.  A call that times out (RRS_ERR_TIMEOUT) may leave
+ * the barrier state dirty: zero-fill the header before using the workspace
+ * again. */
 size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned flags);
 
 /* Offline weight path (summary page "Approach"; rebuttal page "Description of
@@ -185,19 +204,20 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t *qX, const uint8_t *qW, in
                                         int G, int32_t *P, void *ws, size_t ws_bytes, unsigned flags,
                                         rrs_stream_t stream);
 
-/* Weight operand for the tensor cores, written once per layer after
- * rrs_prepare_weights: qW8[n][k'] = 16 * q, where q is the signed INT4 code
- * that qW packs, laid out in the GEMM's k order (within each 8 codes: the
- * even k, then the odd k).  The pages have no counterpart: the INT4 codes
- * themselves are unchanged, only stored one per byte so that the GEMM needs
- * no unpacking step on the chip.  It doubles the weight bytes (N * K instead
- * of N * K / 2) and makes the GEMM faster where it is compute-bound (prefill;
- * pass RRS_W_EXPANDED).  qW packed [N, K/2] as rrs_prepare_weights writes it;
- * qW8 [N, K] device, caller-owned, 16-byte aligned.  K as for rrs_w4a4_gemm.
- * Asynchronous on `stream`.  Errors: RRS_ERR_INVALID_ARG for a null or misaligned
- * pointer or N < 1; RRS_ERR_UNSUPPORTED for K % 128 != 0; RRS_ERR_CUDA if the launch
- * fails. */
-rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, int8_t *qW8, rrs_stream_t stream);
+/* Weight operand of the fp8 tensor-core GEMM, written once per layer after
+ * rrs_prepare_weights: qW8[n][k] = the INT4 code q of qW[n][k] as an e4m3 byte
+ * (natural k order; every code in [-8, 7] is an e4m3 number exactly, and so is
+ * every product of two codes, which the fp32 accumulators of the MMA sum
+ * without rounding).  The pages have no counterpart: the INT4 codes are
+ * unchanged, only stored one per byte in a form the fp8 MMA reads, so that the
+ * per-group promotion of the GEMM is one fused multiply-add on an fp32 partial
+ * sum.  It doubles the weight bytes (N * K instead of N * K / 2); pass
+ * RRS_W_EXPANDED to use it.  qW packed [N, K/2] as rrs_prepare_weights writes it;
+ * qW8 [N, K] bytes, device, caller-owned, 16-byte aligned.  K as for
+ * rrs_w4a4_gemm.  Asynchronous on `stream`.  Errors: RRS_ERR_INVALID_ARG for a
+ * null or misaligned pointer or N < 1; RRS_ERR_UNSUPPORTED for K % 128 != 0;
+ * RRS_ERR_CUDA if the launch fails. */
+rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, uint8_t *qW8, rrs_stream_t stream);
 
 /* Gated-MLP step between two RRS linears (summary page "Key results": the method is
  * applied to every linear layer of the model, so the down projection's input is the

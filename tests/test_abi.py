@@ -172,3 +172,14 @@ def test_product_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "rrs_oracle" not in src, f
+
+
+def test_interleave_gate_up_rows_without_gpu():
+    import torch
+    from activation_smoothing_b200 import _binding as b
+    Wg = torch.arange(12, dtype=torch.float32).reshape(3, 4)
+    Wu = -Wg
+    W = b.interleave_gate_up(Wg, Wu)
+    assert W.shape == (6, 4)
+    assert torch.equal(W[0::2], Wg) and torch.equal(W[1::2], Wu)
+    assert b._y_shape(8, 10, b.Y_SILU_MUL) == (8, 5) and b._y_dtype(b.Y_SILU_MUL) == torch.float16

@@ -121,3 +121,36 @@ def test_mlp_block_quality_bounded(rrs):
         errs[name] = (torch.linalg.vector_norm(Y - ref) / torch.linalg.vector_norm(ref)).item()
     print("mlp block relative error vs fp32:", errs)
     assert all(np.isfinite(v) and v < 0.5 for v in errs.values()), errs
+
+
+@pytest.mark.parametrize("M,F,K", [(512, 9472, 512), (130, 260, 256), (64, 1000, 384)])
+def test_gate_up_gemm_with_fused_silu_mul(rrs, M, F, K):
+    """RRS_Y_SILU_MUL: the fp8 gate/up GEMM over interleaved weight rows writes H directly;
+    it must equal, bit for bit, rrs_silu_mul applied to the same GEMM's fp32 output with
+    its columns de-interleaved into [gate | up] (the shapes take the CTA-pair kernel and
+    the single-CTA one, with ragged edges)."""
+    G = 128
+    rng = np.random.default_rng(M + F)
+    qX = torch.from_numpy(rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)).to(DEV)
+    qW = torch.from_numpy(rng.integers(0, 256, size=(2 * F, K // 2), dtype=np.uint8)).to(DEV)
+    s = torch.from_numpy((rng.random(K // G, dtype=np.float32) + 0.5).astype(np.float32)).to(DEV)
+    st = torch.from_numpy((rng.random(M, dtype=np.float32) * 0.05).astype(np.float32)).to(DEV)
+    sw = torch.from_numpy((rng.random(2 * F, dtype=np.float32) * 0.05).astype(np.float32)).to(DEV)
+    qW8 = rrs.expand_weights(qW)
+    Y = rrs.w4a4_gemm(qX, s, st, qW8, sw, G, flags=rrs.W_EXPANDED)
+    H = rrs.w4a4_gemm(qX, s, st, qW8, sw, G, flags=rrs.W_EXPANDED | rrs.Y_SILU_MUL)
+    GU = torch.cat([Y[:, 0::2], Y[:, 1::2]], dim=1).contiguous()
+    Href = rrs.silu_mul(GU)
+    torch.cuda.synchronize()
+    assert H.shape == (M, F) and H.dtype == torch.float16
+    assert torch.equal(H.view(torch.int16), Href.view(torch.int16))
+
+
+def test_silu_mul_flag_needs_the_fp8_path(rrs):
+    qX = torch.zeros(4, 128, dtype=torch.uint8, device=DEV)
+    qW = torch.zeros(8, 128, dtype=torch.uint8, device=DEV)
+    s = torch.ones(2, device=DEV)
+    with pytest.raises(rrs.RRSError) as e:
+        rrs.w4a4_gemm(qX, s, torch.ones(4, device=DEV), qW, torch.ones(8, device=DEV), 128, flags=rrs.Y_SILU_MUL)
+    assert e.value.status_name == "RRS_ERR_UNSUPPORTED"
+
