@@ -42,6 +42,8 @@ def lib() -> ctypes.CDLL:
         L.orc_group_partials.argtypes = [P, P, i64, i64, i32, i32, P, i64, P]
         L.orc_linear_rows.argtypes = [P, P, P, P, P, i64, i64, i32, i32, P, i64, P, P]
         L.orc_channel_absmax.argtypes = [P, i64, i32, i32, P]
+        L.orc_kv_quant.argtypes = [P, i64, i32, P, P, P]
+        L.orc_kv_dequant.argtypes = [P, i64, i32, P, P]
         _lib = L
     return _lib
 
@@ -231,3 +233,31 @@ def silu_mul(GU) -> np.ndarray:
     g, u = gu[:, :F], gu[:, F:]
     h = g / (1.0 + np.exp(-g)) * u
     return np.clip(h, -65504.0, 65504.0).astype(np.float16)
+
+
+def kv_quant(KV):
+    """KV-cache quantisation (the 4-4-4 setting) of fp16/fp32 KV [..., D]: every head
+    vector rotated by the normalised Hadamard transform of size D, then per-vector
+    symmetric INT4.  -> (codes int8 [..., D], q uint8 [..., D/2], scale fp32 [...])."""
+    x = _f32(KV)
+    lead = x.shape[:-1]
+    D = x.shape[-1]
+    x2 = np.ascontiguousarray(x.reshape(-1, D))
+    rows = x2.shape[0]
+    codes = np.empty((rows, D), np.int8)
+    q = np.empty((rows, D // 2), np.uint8)
+    scale = np.empty(rows, np.float32)
+    _check(lib().orc_kv_quant(_p(x2), rows, D, _p(codes), _p(q), _p(scale)), "kv_quant")
+    return codes.reshape(*lead, D), q.reshape(*lead, D // 2), scale.reshape(lead)
+
+
+def kv_dequant(q, scale) -> np.ndarray:
+    """code * scale in fp32, in the rotated space: q uint8 [..., D/2], scale [...] -> [..., D]."""
+    qq = np.ascontiguousarray(np.asarray(q, np.uint8))
+    lead = qq.shape[:-1]
+    D = 2 * qq.shape[-1]
+    q2 = qq.reshape(-1, D // 2)
+    sc = np.ascontiguousarray(np.asarray(scale, np.float32).reshape(-1))
+    out = np.empty((q2.shape[0], D), np.float32)
+    _check(lib().orc_kv_dequant(_p(q2), q2.shape[0], D, _p(sc), _p(out)), "kv_dequant")
+    return out.reshape(*lead, D)

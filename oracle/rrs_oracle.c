@@ -38,6 +38,9 @@
  *  R6  4-bit symmetric quantiser: scale = amax / 7 (q_A = 7), fp32.
  *  R7  round half to even (rintf in the default rounding mode).
  *  R8  no clipping ratio.
+ *  R14 KV cache (the "4-4-4" setting): each head vector rotated by the
+ *      normalised Hadamard transform of its length D, then the per-token
+ *      symmetric INT4 quantiser; no runtime smoothing (see orc_kv_quant).
  *  R9  packing: byte i = (q[2i] & 0xF) | (q[2i+1] & 0xF) << 4, two's
  *      complement nibbles.
  *  Y   sum_g s_g * P_g accumulated in double, times scale_t and scale_w in
@@ -310,5 +313,45 @@ int orc_channel_absmax(const float *X, int64_t M, int K, int n, float *cmax)
         }
     }
     free(rot);
+    return 0;
+}
+
+/* KV-cache quantisation of the "4-4-4" setting ([RRS-summary] "Key results":
+ * weights, activations and the KV cache held in 4 bits).  Reading R14: every
+ * head vector of K or V (length D, one row here) is rotated by the normalised
+ * Hadamard transform of size D (the rotation of R1-R2 with n = D) and then
+ * quantised by the per-token symmetric INT4 quantiser (quant_row; readings
+ * R4, R6-R9).  There is no runtime smoothing: the runtime group scales belong to
+ * the linear layer's group-scaled GEMM, which the attention products lack.
+ * KV fp32 [rows, D] -> codes int8 [rows, D] (optional, may be NULL), packed
+ * q [rows, D/2], scale [rows]. */
+int orc_kv_quant(const float *KV, int64_t rows, int D, int8_t *codes, uint8_t *q, float *scale)
+{
+    if (!is_pow2(D) || D < 2) return -1;
+    float *rot = (float *)malloc(sizeof(float) * (size_t)D);
+    int8_t *c = (int8_t *)malloc((size_t)D);
+    int rc = 0;
+    if (!rot || !c) { rc = -2; goto done; }
+    for (int64_t r = 0; r < rows; ++r) {
+        rc = orc_rotate(KV + r * (int64_t)D, 1, D, D, rot);
+        if (rc) goto done;
+        scale[r] = quant_row(rot, D, c);
+        if (codes) memcpy(codes + r * (int64_t)D, c, (size_t)D);
+        pack_row(c, D, q + r * (int64_t)(D / 2));
+    }
+done:
+    free(rot);
+    free(c);
+    return rc;
+}
+
+/* The cached vector back in the rotated space: x_hat = code * scale in fp32
+ * (the quantiser's own reconstruction, [L2Rot] Sec. 3.1: Delta * round(Z / Delta)). */
+int orc_kv_dequant(const uint8_t *q, int64_t rows, int D, const float *scale, float *out)
+{
+    if (D < 2 || D % 2 != 0) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int j = 0; j < D; ++j)
+            out[r * (int64_t)D + j] = (float)nib(q + r * (int64_t)(D / 2), j) * scale[r];
     return 0;
 }
