@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         "rrs_expand_weights": ([P, I, I, P, P], I),
         "rrs_silu_mul": ([P, I, I, P, P], I),
         "rrs_channel_absmax": ([P, I, I, I, P, U, P], I),
+        "rrs_kv_quant": ([P, I, I, I, P, P, U, P], I),
+        "rrs_kv_dequant": ([P, P, I, I, I, P, P], I),
         "rrs_perm_from_channel_max": ([P, I, P], I),
         "rrs_check_workspace": ([P, P], I),
         "rrs_debug_wait_timeout": ([I, P, Z, P], I),
@@ -325,6 +327,33 @@ def expand_weights(qW: torch.Tensor, qW8: Optional[torch.Tensor] = None, stream=
     _need(qW8, "qW8", torch.float8_e4m3fn, (N, K))
     _check(lib().rrs_expand_weights(_ptr(qW), N, K, _ptr(qW8), _stream(stream)))
     return qW8
+
+
+def kv_quant(KV: torch.Tensor, q: Optional[torch.Tensor] = None, scale: Optional[torch.Tensor] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """KV cache (4-4-4 setting): fp16 KV [T, H, D] -> (q uint8 [T, H, D/2], scale fp32 [T, H]),
+    every head vector rotated by the normalised Hadamard transform of size D."""
+    T, H, D = KV.shape
+    _need(KV, "KV", torch.float16, (T, H, D))
+    q = torch.empty((T, H, D // 2), dtype=torch.uint8, device=KV.device) if q is None else q
+    scale = torch.empty((T, H), dtype=torch.float32, device=KV.device) if scale is None else scale
+    _need(q, "q", torch.uint8, (T, H, D // 2))
+    _need(scale, "scale", torch.float32, (T, H))
+    _check(lib().rrs_kv_quant(_ptr(KV), T, H, D, _ptr(q), _ptr(scale), 0, _stream(stream)))
+    return q, scale
+
+
+def kv_dequant(q: torch.Tensor, scale: torch.Tensor, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """fp16 [T, H, D] = code * scale, in the rotated space."""
+    T, H, D2 = q.shape
+    D = 2 * D2
+    _need(q, "q", torch.uint8, (T, H, D2))
+    _need(scale, "scale", torch.float32, (T, H))
+    out = torch.empty((T, H, D), dtype=torch.float16, device=q.device) if out is None else out
+    _need(out, "out", torch.float16, (T, H, D))
+    _check(lib().rrs_kv_dequant(_ptr(q), _ptr(scale), T, H, D, _ptr(out), _stream(stream)))
+    return out
 
 
 def channel_absmax(X: torch.Tensor, had_block: int, flags: int = 0, cmax: Optional[torch.Tensor] = None,

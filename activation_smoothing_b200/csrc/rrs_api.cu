@@ -510,6 +510,45 @@ rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, uint8_t* qW8, rrs
     return RRS_OK;
 }
 
+rrs_status rrs_kv_quant(const void* KV, int T, int H, int D, uint8_t* q, float* scale, unsigned flags,
+                        rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(KV);
+    RRS_REQUIRE_PTR(q);
+    RRS_REQUIRE_PTR(scale);
+    if (T < 1 || H < 1) return fail(RRS_ERR_INVALID_ARG, "T = %d, H = %d", T, H);
+    if (D < 1 || (D & (D - 1)) != 0) return fail(RRS_ERR_INVALID_ARG, "D = %d is not a power of two", D);
+    if (D < 128 || D > kMaxHadamard)
+        return fail(RRS_ERR_UNSUPPORTED, "D = %d: the CUDA path takes head sizes 128..%d", D, kMaxHadamard);
+    if (flags != 0) return fail(RRS_ERR_INVALID_ARG, "rrs_kv_quant takes no flags (got 0x%x)", flags);
+    rrs::PrepLaunch pl{};
+    pl.X = KV;
+    pl.rows = T * H;
+    pl.K = D;
+    pl.n = D;
+    pl.G = D;
+    pl.c_n = (float)(1.0 / std::sqrt((double)D));
+    pl.perm = nullptr;           // no reorder
+    pl.mode = 0;
+    pl.unit_scales = 1;          // no runtime smoothing
+    pl.q_out = q;
+    pl.scale_out = scale;
+    cudaError_t e = rrs::launch_prep(pl, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "KV quantise kernel");
+    return RRS_OK;
+}
+
+rrs_status rrs_kv_dequant(const uint8_t* q, const float* scale, int T, int H, int D, void* out,
+                          rrs_stream_t stream) {
+    RRS_REQUIRE_PTR(q);
+    RRS_REQUIRE_PTR(scale);
+    RRS_REQUIRE_PTR(out);
+    if (T < 1 || H < 1) return fail(RRS_ERR_INVALID_ARG, "T = %d, H = %d", T, H);
+    if (D < 8 || D % 8 != 0) return fail(RRS_ERR_INVALID_ARG, "D = %d is not a positive multiple of 8", D);
+    cudaError_t e = rrs::launch_kv_dequant(q, scale, (size_t)T * H, D, out, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "KV dequantise kernel");
+    return RRS_OK;
+}
+
 rrs_status rrs_channel_absmax(const void* X, int M, int K, int had_block, float* cmax, unsigned flags,
                               rrs_stream_t stream) {
     RRS_REQUIRE_PTR(X);

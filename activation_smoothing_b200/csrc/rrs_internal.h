@@ -81,6 +81,9 @@ struct PrepFastLaunch {
 bool prep_fast_supported(int K, int n);
 int prep_fast_rows_per_cta(int K);
 cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t stream);
+// KV cache: out fp16 [rows, D] = code * scale[row] from packed INT4 q [rows, D/2].
+cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows, int D, void* out,
+                              cudaStream_t stream);
 // p[0..n) = v.
 cudaError_t launch_fill(float* p, int n, float v, cudaStream_t stream);
 // Packed INT4 rows -> int8 rows in the GEMM's k order.

@@ -215,8 +215,9 @@ __global__ void __launch_bounds__(MAXT) prep_kernel(PrepArgs p) {
 #pragma unroll
         for (int l = 0; l < E; l += 2) {
             const int j = t * E + l;
-            const uint32_t lo16 = (uint32_t)swz<LOGE>(p.perm[j]);
-            const uint32_t hi16 = (uint32_t)swz<LOGE>(p.perm[j + 1]);
+            // a null index means no reorder (the KV-cache path)
+            const uint32_t lo16 = (uint32_t)swz<LOGE>(p.perm ? p.perm[j] : j);
+            const uint32_t hi16 = (uint32_t)swz<LOGE>(p.perm ? p.perm[j + 1] : j + 1);
             gaddr[l / 2] = lo16 | (hi16 << 16);
         }
         if (!p.unit_scales) {
@@ -423,7 +424,7 @@ __global__ void __launch_bounds__(MAXT) prep_kernel(PrepArgs p) {
     // scaling the max equals the max of the scaled values).
     for (int j0 = 0; j0 < K; j0 += blockDim.x) {
         const int j = j0 + threadIdx.x;
-        float m = (j < K) ? __uint_as_float(cm[p.perm[j]]) : 0.0f;
+        float m = (j < K) ? __uint_as_float(cm[p.perm ? p.perm[j] : j]) : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0 && j < K && m > 0.0f)

@@ -607,6 +607,11 @@ static cudaError_t launch_act(const ActArgs& a, int threads, size_t smem, int gr
     int grid = (a.rows + R - 1) / R;
     if (grid > occ * nsm) grid = occ * nsm;
     if (grid > grid_cap) grid = grid_cap;
+    if (!(a.phase & 1)) {
+        // quantisation alone (given scales): no grid-wide barrier, a plain launch
+        kern<<<grid, threads, smem, st>>>(a);
+        return cudaGetLastError();
+    }
     ActArgs args = a;
     void* params[] = {&args};
     // all CTAs must be resident together: the phases meet at a grid-wide barrier

@@ -230,6 +230,28 @@ rrs_status rrs_expand_weights(const uint8_t *qW, int N, int K, uint8_t *qW8, rrs
  * pointer or M, F < 1; RRS_ERR_CUDA if the launch fails. */
 rrs_status rrs_silu_mul(const float *GU, int M, int F, void *H, rrs_stream_t stream);
 
+/* KV cache of the 4-4-4 setting (summary page, "Key results": weights,
+ * activations and the KV cache in 4 bits).  Reading: every head vector of K or
+ * V (length D) is rotated by the normalised Hadamard transform of size D (the
+ * same fp32 stage order and c_D as the activations) and quantised to
+ * symmetric INT4 with its own scale, scale = max |x_rot| / 7, code =
+ * clamp(rint(x_rot / scale), -8, 7), no reorder and no runtime smoothing (the
+ * runtime group scales belong to the linear layer's GEMM).  A query rotated by
+ * the same transform gives the same attention scores (the transform is
+ * orthogonal).  KV fp16 [T, H, D] (token, head, channel), q uint8 [T, H, D/2]
+ * (low nibble = even channel), scale fp32 [T, H]; device, caller-owned,
+ * 16-byte aligned.  D a power of two, 128 <= D <= 8192 on the CUDA path
+ * (RRS_ERR_UNSUPPORTED otherwise); flags must be 0.  Asynchronous on `stream`;
+ * no workspace. */
+rrs_status rrs_kv_quant(const void *KV, int T, int H, int D, uint8_t *q, float *scale, unsigned flags,
+                        rrs_stream_t stream);
+
+/* The cached vectors back, in the rotated space: out fp16 [T, H, D] =
+ * fp16(code * scale) (the product in fp32, then rounded to nearest even).
+ * D a positive multiple of 8.  Asynchronous on `stream`. */
+rrs_status rrs_kv_dequant(const uint8_t *q, const float *scale, int T, int H, int D, void *out,
+                          rrs_stream_t stream);
+
 /* Calibration statistic for the reorder index: cmax[k] = max_t |X_rot[t][k]|
  * (rotation only, no reorder).  cmax fp32 [K]. */
 rrs_status rrs_channel_absmax(const void *X, int M, int K, int had_block, float *cmax,

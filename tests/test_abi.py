@@ -105,6 +105,14 @@ def test_argument_checks_fail_before_any_launch(L):
     # the scales come from s: unit scales do not apply to pass B
     assert L.rrs_smooth_quant_scaled(ok, 16, 256, 128, 256, ok, ok, ok, ok, ws, 1 << 20, 2, None) == 1
     assert b"s filled with 1" in L.rrs_last_error_string()
+    # KV cache: null pointers, bad sizes, flags
+    assert L.rrs_kv_quant(None, 4, 2, 128, ok, ok, 0, None) == 1
+    assert L.rrs_kv_quant(ok, 0, 2, 128, ok, ok, 0, None) == 1
+    assert L.rrs_kv_quant(ok, 4, 2, 96, ok, ok, 0, None) == 1        # not a power of two
+    assert L.rrs_kv_quant(ok, 4, 2, 64, ok, ok, 0, None) == 2        # below the CUDA path's head size
+    assert L.rrs_kv_quant(ok, 4, 2, 128, ok, ok, 1, None) == 1       # no flags
+    assert L.rrs_kv_dequant(ok, ok, 4, 2, 12, ok, None) == 1
+    assert L.rrs_kv_dequant(ok, None, 4, 2, 128, ok, None) == 1
     # M < 1
     assert L.rrs_w4a4_gemm(ok, ok, ok, ok, ok, 0, 16, 256, 128, ok, ws, 1 << 20, 0, None) == 1
     assert L.rrs_debug_wait_timeout(0, ws, 256, None) == 1
