@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
         "rrs_kv_dequant": ([P, P, I, I, I, P, P], I),
         "rrs_perm_from_channel_max": ([P, I, P], I),
         "rrs_check_workspace": ([P, P], I),
+        "rrs_check_perm": ([P, I, P, Z, P], I),
         "rrs_debug_wait_timeout": ([I, P, Z, P], I),
         "rrs_debug_divide": ([P, P, I, P, P, P], I),
         "rrs_last_error_string": ([], ctypes.c_char_p),
@@ -385,6 +386,16 @@ def calibrate_perm(X_cal: torch.Tensor, had_block: int, flags: int = 0) -> torch
 def check_workspace(ws: torch.Tensor, stream=None) -> None:
     """Synchronise and raise RRSError(RRS_ERR_TIMEOUT) if a kernel gave up on a wait."""
     _check(lib().rrs_check_workspace(_ptr(ws), _stream(stream)))
+
+
+def check_perm(perm: torch.Tensor, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Raise RRSError(RRS_ERR_INVALID_ARG) unless the device int32 index perm [K] is a
+    permutation of 0..K-1 (synchronises the stream)."""
+    K = perm.numel()
+    _need(perm, "perm", torch.int32, (K,))
+    if ws is None:
+        ws = torch.empty(256 + 16 + 4 * ((K + 31) // 32), dtype=torch.uint8, device=perm.device)
+    _check(lib().rrs_check_perm(_ptr(perm), K, _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def debug_wait_timeout(limit_us: int, ws: torch.Tensor, stream=None) -> None:

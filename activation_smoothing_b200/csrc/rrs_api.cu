@@ -1,8 +1,9 @@
 // rrs_api.cu -- the extern "C" entry points declared in include/rrs.h:
 // argument validation on the host, then stream-ordered kernel launches.
-// No entry point allocates memory; only rrs_check_workspace and
-// rrs_linear_from_host synchronise the host.
+// No entry point allocates memory; only rrs_check_workspace, rrs_check_perm
+// and rrs_linear_from_host synchronise the host.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -32,6 +33,14 @@ rrs_status fail(rrs_status st, const char* fmt, ...) {
 rrs_status cuda_fail(cudaError_t e, const char* what) {
     return fail(RRS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
+
+// One NVTX range per entry point, named after it, for timeline tools; without
+// a tool attached the push and pop return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+#define RRS_TRACE() NvtxRange rrs_trace_range_(__func__)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -314,6 +323,7 @@ size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned fl
 
 rrs_status rrs_prepare_weights(const void* W, int N, int K, int had_block, const int32_t* perm, uint8_t* qW,
                                float* scale_w, unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(W);
     RRS_REQUIRE_PTR(perm);
     RRS_REQUIRE_PTR(qW);
@@ -345,6 +355,7 @@ rrs_status rrs_prepare_weights(const void* W, int N, int K, int had_block, const
 rrs_status rrs_smooth_quant(const void* X, int M, int K, int G, int had_block, const int32_t* perm, uint8_t* qX,
                             float* s, float* scale_t, void* ws, size_t ws_bytes, unsigned flags,
                             rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(X);
     RRS_REQUIRE_PTR(perm);
     RRS_REQUIRE_PTR(qX);
@@ -367,6 +378,7 @@ rrs_status rrs_smooth_quant(const void* X, int M, int K, int G, int had_block, c
 
 rrs_status rrs_group_max(const void* X, int M, int K, int G, int had_block, const int32_t* perm, float* s,
                          void* ws, size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(X);
     RRS_REQUIRE_PTR(perm);
     RRS_REQUIRE_PTR(s);
@@ -394,6 +406,7 @@ rrs_status rrs_group_max(const void* X, int M, int K, int G, int had_block, cons
 rrs_status rrs_smooth_quant_scaled(const void* X, int M, int K, int G, int had_block, const int32_t* perm,
                                    const float* s, uint8_t* qX, float* scale_t, void* ws, size_t ws_bytes,
                                    unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(X);
     RRS_REQUIRE_PTR(perm);
     RRS_REQUIRE_PTR(s);
@@ -420,6 +433,7 @@ rrs_status rrs_smooth_quant_scaled(const void* X, int M, int K, int G, int had_b
 rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t, const uint8_t* qW,
                          const float* scale_w, int M, int N, int K, int G, float* Y, void* ws, size_t ws_bytes,
                          unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(qX);
     RRS_REQUIRE_PTR(s);
     RRS_REQUIRE_PTR(scale_t);
@@ -445,6 +459,7 @@ rrs_status rrs_w4a4_gemm(const uint8_t* qX, const float* s, const float* scale_t
 rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, const int32_t* perm, int M, int N,
                       int K, int G, int had_block, uint8_t* qX, float* s, float* scale_t, float* Y, void* ws,
                       size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
     return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes,
@@ -455,6 +470,7 @@ rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* 
                                 const int32_t* perm, int M, int N, int K, int G, int had_block, uint8_t* qX,
                                 float* s, float* scale_t, float* Y_dev, float* Y_host, void* ws,
                                 size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     if (X_host == nullptr || Y_host == nullptr) return fail(RRS_ERR_INVALID_ARG, "host buffer is null");
     RRS_REQUIRE_PTR(X_dev);
     RRS_REQUIRE_PTR(Y_dev);
@@ -476,6 +492,7 @@ rrs_status rrs_linear_from_host(const void* X_host, void* X_dev, const uint8_t* 
 rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, int M, int N, int K, int G,
                                         int32_t* P, void* ws, size_t ws_bytes, unsigned flags,
                                         rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(qX);
     RRS_REQUIRE_PTR(qW);
     RRS_REQUIRE_PTR(P);
@@ -491,6 +508,7 @@ rrs_status rrs_w4a4_gemm_debug_partials(const uint8_t* qX, const uint8_t* qW, in
 }
 
 rrs_status rrs_silu_mul(const float* GU, int M, int F, void* H, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(GU);
     RRS_REQUIRE_PTR(H);
     if (M < 1 || F < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, F = %d", M, F);
@@ -500,6 +518,7 @@ rrs_status rrs_silu_mul(const float* GU, int M, int F, void* H, rrs_stream_t str
 }
 
 rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, uint8_t* qW8, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(qW);
     RRS_REQUIRE_PTR(qW8);
     if (N < 1) return fail(RRS_ERR_INVALID_ARG, "N = %d", N);
@@ -512,6 +531,7 @@ rrs_status rrs_expand_weights(const uint8_t* qW, int N, int K, uint8_t* qW8, rrs
 
 rrs_status rrs_kv_quant(const void* KV, int T, int H, int D, uint8_t* q, float* scale, unsigned flags,
                         rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(KV);
     RRS_REQUIRE_PTR(q);
     RRS_REQUIRE_PTR(scale);
@@ -539,6 +559,7 @@ rrs_status rrs_kv_quant(const void* KV, int T, int H, int D, uint8_t* q, float* 
 
 rrs_status rrs_kv_dequant(const uint8_t* q, const float* scale, int T, int H, int D, void* out,
                           rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(q);
     RRS_REQUIRE_PTR(scale);
     RRS_REQUIRE_PTR(out);
@@ -549,8 +570,32 @@ rrs_status rrs_kv_dequant(const uint8_t* q, const float* scale, int T, int H, in
     return RRS_OK;
 }
 
+rrs_status rrs_check_perm(const int32_t* perm, int K, void* ws, size_t ws_bytes, rrs_stream_t stream) {
+    RRS_TRACE();
+    RRS_REQUIRE_PTR(perm);
+    if (K < 1) return fail(RRS_ERR_INVALID_ARG, "K = %d", K);
+    const size_t need = kHeaderBytes + rrs::perm_check_bytes(K);
+    rrs_status r = check_ws(ws, ws_bytes, need);
+    if (r != RRS_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned char* scratch = static_cast<unsigned char*>(ws) + kHeaderBytes;
+    cudaError_t e = rrs::launch_perm_check(perm, K, scratch, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reorder-index check kernels");
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t words[2] = {0, 0};
+    e = cudaMemcpy(words, scratch, sizeof(words), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the check result");
+    if (words[0] < (uint32_t)K)
+        return fail(RRS_ERR_INVALID_ARG, "perm[%u] is outside [0, %d)", words[0], K);
+    if (words[1] < (uint32_t)K)
+        return fail(RRS_ERR_INVALID_ARG, "perm is not a permutation: no position holds %u", words[1]);
+    return RRS_OK;
+}
+
 rrs_status rrs_channel_absmax(const void* X, int M, int K, int had_block, float* cmax, unsigned flags,
                               rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(X);
     RRS_REQUIRE_PTR(cmax);
     if (M < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d", M);
@@ -578,6 +623,7 @@ rrs_status rrs_channel_absmax(const void* X, int M, int K, int had_block, float*
 }
 
 rrs_status rrs_perm_from_channel_max(const float* cmax_host, int K, int32_t* perm_host) {
+    RRS_TRACE();
     if (cmax_host == nullptr || perm_host == nullptr) return fail(RRS_ERR_INVALID_ARG, "null host buffer");
     if (K < 1) return fail(RRS_ERR_INVALID_ARG, "K = %d", K);
     std::vector<int32_t> idx((size_t)K);
@@ -589,6 +635,7 @@ rrs_status rrs_perm_from_channel_max(const float* cmax_host, int K, int32_t* per
 }
 
 rrs_status rrs_check_workspace(void* ws, rrs_stream_t stream) {
+    RRS_TRACE();
     if (ws == nullptr) return fail(RRS_ERR_WORKSPACE, "workspace is null");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);
@@ -606,6 +653,7 @@ rrs_status rrs_check_workspace(void* ws, rrs_stream_t stream) {
 }
 
 rrs_status rrs_debug_wait_timeout(int limit_us, void* ws, size_t ws_bytes, rrs_stream_t stream) {
+    RRS_TRACE();
     rrs_status r = check_ws(ws, ws_bytes, kHeaderBytes);
     if (r != RRS_OK) return r;
     if (limit_us < 1 || limit_us > 1000000) return fail(RRS_ERR_INVALID_ARG, "limit_us = %d", limit_us);
@@ -617,6 +665,7 @@ rrs_status rrs_debug_wait_timeout(int limit_us, void* ws, size_t ws_bytes, rrs_s
 
 rrs_status rrs_debug_divide(const float* a, const float* b, int n, float* q_fast, float* q_ieee,
                             rrs_stream_t stream) {
+    RRS_TRACE();
     if (!a || !b || !q_fast || !q_ieee || n < 1) return fail(RRS_ERR_INVALID_ARG, "rrs_debug_divide arguments");
     cudaError_t e = rrs::launch_divide_check(a, b, n, q_fast, q_ieee, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "divide check kernel");
@@ -625,6 +674,7 @@ rrs_status rrs_debug_divide(const float* a, const float* b, int n, float* q_fast
 
 rrs_status rrs_smooth_quant_noalloc(const void* X, int M, int K, int G, int had_block, const int32_t* perm,
                                     uint8_t* qX, float* s, float* scale_t, unsigned flags, rrs_stream_t stream) {
+    RRS_TRACE();
     RRS_REQUIRE_PTR(X);
     RRS_REQUIRE_PTR(perm);
     RRS_REQUIRE_PTR(qX);

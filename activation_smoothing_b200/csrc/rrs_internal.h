@@ -86,6 +86,11 @@ cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows,
                               cudaStream_t stream);
 // p[0..n) = v.
 cudaError_t launch_fill(float* p, int n, float v, cudaStream_t stream);
+// Reorder-index check (rrs_check.cu): scratch of perm_check_bytes(K) bytes;
+// words 0 and 1 of it receive the first out-of-range position and the smallest
+// missing value (K when there is none).
+size_t perm_check_bytes(int K);
+cudaError_t launch_perm_check(const int32_t* perm, int K, void* scratch, cudaStream_t stream);
 // Packed INT4 rows -> int8 rows in the GEMM's k order.
 cudaError_t launch_expand(const uint8_t* qX, int8_t* qX8, int M, int K, cudaStream_t stream);
 

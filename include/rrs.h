@@ -44,7 +44,8 @@
  *
  * Ownership: the caller owns every buffer, including the workspace.  The
  * library allocates no device or host memory and never synchronises the host
- * except in rrs_check_workspace and rrs_linear_from_host (documented there).
+ * except in rrs_check_workspace, rrs_check_perm and rrs_linear_from_host
+ * (documented there).
  * Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  * and outputs are valid when the stream reaches that point.  Calls that share
  * output buffers or a workspace must be ordered on one stream.
@@ -265,6 +266,17 @@ rrs_status rrs_perm_from_channel_max(const float *cmax_host, int K, int32_t *per
  * Returns RRS_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
  * last check, RRS_OK otherwise. */
 rrs_status rrs_check_workspace(void *ws, rrs_stream_t stream);
+
+/* Debug check of the reorder index (rebuttal page, "Description of the
+ * reorder process": the reorder permutes channels).  The hot path trusts perm;
+ * this entry checks that perm (device, int32 [K]) holds every value of
+ * 0..K-1 exactly once.  Uses ws past its 256-byte header as scratch (needs
+ * ws_bytes >= 256 + 16 + 4 * ceil(K / 32); any workspace sized by
+ * rrs_workspace_size for this K is enough), then synchronises `stream` and
+ * reads the result.  Returns RRS_OK, or RRS_ERR_INVALID_ARG naming the first
+ * position whose value is out of range, else the smallest value no position
+ * holds (which, with K in-range entries, means another value is repeated). */
+rrs_status rrs_check_perm(const int32_t *perm, int K, void *ws, size_t ws_bytes, rrs_stream_t stream);
 
 /* Fault-injection hook for tests: launches one kernel that waits on a
  * barrier nothing will release, with a wait limit of `limit_us`

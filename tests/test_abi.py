@@ -136,6 +136,23 @@ def test_next_row_entry_points_check_arguments_before_any_launch(L):
     assert L.rrs_expand_weights(ok, 16, 200, ok, None) == 2     # K % 128 != 0: unsupported
 
 
+def test_check_perm_checks_arguments_before_any_launch(L):
+    ok = _fake(0x10000)
+    mis = _fake(0x10004)
+    K = 4096
+    need = 256 + 16 + 4 * ((K + 31) // 32)
+    # rrs_check_perm(perm, K, ws, ws_bytes, stream)
+    assert L.rrs_check_perm(None, K, ok, need, None) == 1
+    assert b"perm" in L.rrs_last_error_string()
+    assert L.rrs_check_perm(mis, K, ok, need, None) == 1
+    assert L.rrs_check_perm(ok, 0, ok, need, None) == 1
+    assert L.rrs_check_perm(ok, K, None, need, None) == 5           # workspace missing
+    assert L.rrs_check_perm(ok, K, ok, need - 4, None) == 5         # one bitmap word short
+    assert b"need" in L.rrs_last_error_string()
+    # any workspace rrs_workspace_size gives for this K is large enough
+    assert L.rrs_workspace_size(1, 0, K, 128, K, 0) >= need
+
+
 def test_binding_shape_checks_without_gpu():
     import torch
     import activation_smoothing_b200 as rrs
