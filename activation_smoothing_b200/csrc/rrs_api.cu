@@ -312,6 +312,7 @@ size_t rrs_workspace_size(int M, int N, int K, int G, int had_block, unsigned fl
     if (M < 1 || K < 1) return kHeaderBytes;
     const int n = (flags & RRS_NO_ROTATE) ? 1 : had_block;
     size_t b = ws_bytes_full(M, K, n);
+    if (M <= 16 && N > 0) b = std::max(b, kHeaderBytes + rrs::decode_ws_bytes(M, N, K));
     if (M <= rrs::kSplitRoomMaxM && N > 0) {
         // split-k partial sums share the space after the int8 operand with the scratch
         const size_t room = align256((size_t)rrs::kSplitRoom * M * N * 4);
@@ -460,6 +461,53 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
                       int K, int G, int had_block, uint8_t* qX, float* s, float* scale_t, float* Y, void* ws,
                       size_t ws_bytes, unsigned flags, rrs_stream_t stream) {
     RRS_TRACE();
+    if (M >= 1 && M <= 16 && !(flags & (RRS_W_EXPANDED | RRS_Y_SILU_MUL))) {
+        // few tokens: the whole layer in one launch when the shape and workspace allow
+        RRS_REQUIRE_PTR(X);
+        RRS_REQUIRE_PTR(perm);
+        RRS_REQUIRE_PTR(qX);
+        RRS_REQUIRE_PTR(s);
+        RRS_REQUIRE_PTR(scale_t);
+        RRS_REQUIRE_PTR(qW);
+        RRS_REQUIRE_PTR(scale_w);
+        RRS_REQUIRE_PTR(Y);
+        if (N < 1) return fail(RRS_ERR_INVALID_ARG, "M = %d, N = %d", M, N);
+        rrs_status r = check_K(K);
+        if (r != RRS_OK) return r;
+        r = check_G(K, G);
+        if (r != RRS_OK) return r;
+        int n;
+        float c_n;
+        r = check_hadamard(K, had_block, flags, &n, &c_n);
+        if (r != RRS_OK) return r;
+        r = check_ws(ws, ws_bytes, ws_bytes_full(M, K, n));
+        if (r != RRS_OK) return r;
+        if (ws_bytes >= kHeaderBytes + rrs::decode_ws_bytes(M, N, K) && rrs::decode_supported(M, N, K, G, n)) {
+            rrs::DecodeLaunch dl{};
+            dl.X = X;
+            dl.perm = perm;
+            dl.qW = qW;
+            dl.scale_w = scale_w;
+            dl.M = M;
+            dl.N = N;
+            dl.K = K;
+            dl.G = G;
+            dl.n = n;
+            dl.c_n = c_n;
+            dl.unit_scales = (flags & RRS_FORCE_UNIT_SCALES) ? 1 : 0;
+            dl.qX = qX;
+            dl.s = s;
+            dl.scale_t = scale_t;
+            dl.Y = Y;
+            dl.ybf16 = (flags & RRS_Y_BF16) ? 1 : 0;
+            dl.body = static_cast<unsigned char*>(ws) + kHeaderBytes;
+            dl.gbar = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kBarrierOffset);
+            dl.err = reinterpret_cast<uint32_t*>(ws);
+            cudaError_t e = rrs::launch_decode(dl, reinterpret_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess) return cuda_fail(e, "single-launch linear kernel");
+            return RRS_OK;
+        }
+    }
     rrs_status r = rrs_smooth_quant(X, M, K, G, had_block, perm, qX, s, scale_t, ws, ws_bytes, flags, stream);
     if (r != RRS_OK) return r;
     return rrs_w4a4_gemm(qX, s, scale_t, qW, scale_w, M, N, K, G, Y, ws, ws_bytes,

@@ -186,6 +186,42 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Grid-wide barrier for a cooperative launch: sense reversal on two words
+// (arrival count, generation).  The last CTA to arrive resets the count and
+// advances the generation; the others wait for the generation to change, at
+// most limit_ns, then record a timeout in the error word and report failure.
+__device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t* err, uint64_t limit_ns) {
+    __shared__ int ok_s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        volatile uint32_t* vgen = gbar + 1;
+        const uint32_t gen = *vgen;
+        __threadfence();
+        const uint32_t old = atomicAdd(gbar, 1u);
+        if (old == gridDim.x - 1) {
+            atomicExch(gbar, 0u);
+            __threadfence();
+            atomicAdd(gbar + 1, 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t it = 0;
+            while (*vgen == gen) {
+                if ((++it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+                    atomicOr(err, kErrPrepTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        ok_s = ok;
+    }
+    __syncthreads();
+    return ok_s != 0;
+}
+
 // The gated-MLP activation of one output: silu(g) * u with silu(g) = g / (1 +
 // exp(-g)) in fp32, saturated to +-65504 (the fp16 range the next layer's
 // activation path takes); the caller rounds it to fp16.  One definition for the

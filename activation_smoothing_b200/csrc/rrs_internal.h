@@ -86,6 +86,30 @@ cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows,
                               cudaStream_t stream);
 // p[0..n) = v.
 cudaError_t launch_fill(float* p, int n, float v, cudaStream_t stream);
+// The whole linear layer for M <= 16 tokens in one cooperative launch
+// (rrs_decode.cu).  `body` is the workspace past its 256-byte header, at least
+// decode_ws_bytes(M, N, K) bytes; gbar and err are the header's words.
+struct DecodeLaunch {
+    const void* X;             // fp16 [M, K]
+    const int32_t* perm;
+    const uint8_t* qW;         // packed [N, K/2]
+    const float* scale_w;
+    int M, N, K, G, n;
+    float c_n;
+    int unit_scales;
+    uint8_t* qX;
+    float* s;
+    float* scale_t;
+    void* Y;                   // fp32 or bf16 [M, N]
+    int ybf16;
+    void* body;
+    uint32_t* gbar;
+    uint32_t* err;
+};
+bool decode_supported(int M, int N, int K, int G, int n);
+size_t decode_ws_bytes(int M, int N, int K);
+cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t stream);
+
 // Reorder-index check (rrs_check.cu): scratch of perm_check_bytes(K) bytes;
 // words 0 and 1 of it receive the first out-of-range position and the smallest
 // missing value (K when there is none).

@@ -187,41 +187,6 @@ __device__ __forceinline__ void cp_async_wait_dyn(int pending) {
     else cp_async_wait<0>();
 }
 
-// Grid-wide barrier for a cooperative launch: sense reversal on two words
-// (arrival count, generation).  The last CTA to arrive resets the count and
-// advances the generation; the others wait for the generation to change, at
-// most limit_ns, then record a timeout in the error word and report failure.
-__device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t* err, uint64_t limit_ns) {
-    __shared__ int ok_s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        volatile uint32_t* vgen = gbar + 1;
-        const uint32_t gen = *vgen;
-        __threadfence();
-        const uint32_t old = atomicAdd(gbar, 1u);
-        if (old == gridDim.x - 1) {
-            atomicExch(gbar, 0u);
-            __threadfence();
-            atomicAdd(gbar + 1, 1u);
-        } else {
-            const uint64_t t0 = globaltimer_ns();
-            uint32_t it = 0;
-            while (*vgen == gen) {
-                if ((++it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
-                    atomicOr(err, kErrPrepTimeout);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-        __threadfence();
-        ok_s = ok;
-    }
-    __syncthreads();
-    return ok_s != 0;
-}
 
 // Loads the staged fp16 row into v and runs every butterfly stage of the
 // block Hadamard transform (no scaling).  On return v holds the elements in

@@ -513,6 +513,78 @@ def run_report(args):
         rrs.check_workspace(ws)
         return prep, gemm, Y
 
+    only = args.workload.split(",") if args.workload else None
+    if only is None:
+        run_report_sweep_and_mlp(rrs, wl, dev, out, layer_times)
+    names = ["llama3_8b_down", "llama3_70b_qo", "llama3_70b_gateup", "llama3_70b_down",
+             "llama3_70b_qo_decode_m1", "llama3_70b_qo_decode_m8", "llama3_70b_qo_decode_m16",
+             "llama3_70b_gateup_decode_m1", "llama3_70b_gateup_decode_m16",
+             "llama3_70b_down_decode_m1", "llama3_70b_down_decode_m16"]
+    for nm in only or names:
+        if nm not in wl.LAYERS:
+            continue
+        L = wl.LAYERS[nm]
+        X = wl.make_activations(L).to(dev)
+        W = wl.make_weights(L).to(dev)
+        int8_peak, hbm_peak, _ = peaks()
+        wbytes = L.N * L.K // 2
+        if L.M <= 16:
+            entry = decode_entry(rrs, wl, dev, L, X, W, hbm_peak)
+        else:
+            prep, gemm, _ = layer_times(L, X, W, L.had_block)
+            entry = {"layer": nm, "M": L.M, "K": L.K, "N": L.N, "G": L.G, "n": L.had_block,
+                     "prep_us": round(prep * 1e3, 2), "gemm_us": round(gemm * 1e3, 2),
+                     "TOPS": round(L.ops / ((prep + gemm) * 1e-3) / 1e12, 2),
+                     "gemm_frac_int8_peak": round(L.ops / (gemm * 1e-3) / 1e12 / int8_peak, 4),
+                     "gemm_weight_GBps": round(wbytes / (gemm * 1e-3) / 1e9, 1)}
+        out["layers"].append(entry)
+        del X, W
+        torch.cuda.empty_cache()
+    print(json.dumps(out), flush=True)
+
+
+def decode_entry(rrs, wl, dev, L, X, W, hbm_peak, iters=24):
+    """A decode layer (M <= 16): rrs_linear (one launch) against the two launches
+    (activation kernel, then the GEMM).  Each timed call reads its own copy of the
+    packed weights, enough copies that they exceed L2, so the weight stream comes
+    from HBM as it would in a model's layer sequence."""
+    n = L.had_block
+    perm = wl.random_perm(L.K, 1).to(dev)
+    qW, sw = rrs.prepare_weights(W, perm, n)
+    wbytes = L.N * L.K // 2
+    copies = max(2, min(12, -(-320_000_000 // wbytes)))
+    qWs = [qW] + [qW.clone() for _ in range(copies - 1)]
+    qX = torch.empty((L.M, L.K // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty(L.K // L.G, dtype=torch.float32, device=dev)
+    st = torch.empty(L.M, dtype=torch.float32, device=dev)
+    Y = torch.empty((L.M, L.N), dtype=torch.float32, device=dev)
+    ws = rrs.make_workspace(L.M, L.N, L.K, L.G, n, device=dev)
+    k = [0]
+
+    def nxt():
+        k[0] = (k[0] + 1) % copies
+        return qWs[k[0]]
+
+    one = _time_ms(lambda: rrs.linear(X, nxt(), sw, perm, L.G, n, Y=Y, qX=qX, s=s, scale_t=st, ws=ws), iters)
+    rrs.check_workspace(ws)
+
+    def two_launches():
+        rrs.smooth_quant(X, perm, L.G, n, qX=qX, s=s, scale_t=st, ws=ws)
+        rrs.w4a4_gemm(qX, s, st, nxt(), sw, L.G, Y=Y, ws=ws, flags=rrs.WS_HOLDS_A8)
+
+    two = _time_ms(two_launches, iters)
+    prep = _time_ms(lambda: rrs.smooth_quant(X, perm, L.G, n, qX=qX, s=s, scale_t=st, ws=ws), iters)
+    rrs.check_workspace(ws)
+    gbps = wbytes / (one * 1e-3) / 1e9
+    return {"layer": L.name, "M": L.M, "K": L.K, "N": L.N, "G": L.G, "n": n,
+            "single_launch_us": round(one * 1e3, 2), "two_launches_us": round(two * 1e3, 2),
+            "prep_us": round(prep * 1e3, 2), "weight_copies_rotated": copies,
+            "single_launch_weight_GBps": round(gbps, 1),
+            "single_launch_frac_hbm": round(gbps / hbm_peak, 4),
+            "TOPS": round(L.ops / (one * 1e-3) / 1e12, 3)}
+
+
+def run_report_sweep_and_mlp(rrs, wl, dev, out, layer_times):
     # group-size sweep on the K=4096, N=14336, M=2048 layer
     base = wl.Layer("sweep", 2048, 4096, 14336, 128, 4096, seed=4242)
     X = wl.make_activations(base).to(dev)
@@ -557,28 +629,6 @@ def run_report(args):
                         "TOPS": round((Lgu.ops + Ld.ops) / (total * 1e-3) / 1e12, 1)}
     del Xgu, GU, H
     torch.cuda.empty_cache()
-
-    names = ["llama3_8b_down", "llama3_70b_qo", "llama3_70b_gateup", "llama3_70b_down",
-             "llama3_70b_qo_decode_m1", "llama3_70b_qo_decode_m8", "llama3_70b_qo_decode_m16",
-             "llama3_70b_gateup_decode_m1", "llama3_70b_gateup_decode_m16",
-             "llama3_70b_down_decode_m1", "llama3_70b_down_decode_m16"]
-    for nm in names:
-        if nm not in wl.LAYERS:
-            continue
-        L = wl.LAYERS[nm]
-        X = wl.make_activations(L).to(dev)
-        W = wl.make_weights(L).to(dev)
-        prep, gemm, _ = layer_times(L, X, W, L.had_block)
-        int8_peak, hbm_peak, _ = peaks()
-        wbytes = L.N * L.K // 2
-        out["layers"].append({"layer": nm, "M": L.M, "K": L.K, "N": L.N, "G": L.G, "n": L.had_block,
-                              "prep_us": round(prep * 1e3, 2), "gemm_us": round(gemm * 1e3, 2),
-                              "TOPS": round(L.ops / ((prep + gemm) * 1e-3) / 1e12, 2),
-                              "gemm_frac_int8_peak": round(L.ops / (gemm * 1e-3) / 1e12 / int8_peak, 4),
-                              "gemm_weight_GBps": round(wbytes / (gemm * 1e-3) / 1e9, 1)})
-        del X, W
-        torch.cuda.empty_cache()
-    print(json.dumps(out), flush=True)
 
 
 def main():
