@@ -286,17 +286,21 @@ cudaError_t kernel_setup(const void* kern, int threads, size_t smem, KernelSetup
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const bool cacheable = dev >= 0 && dev < 16;
-    if (cacheable && cache.attr[dev] && cache.occ[dev] > 0) {
+    if (cacheable && cache.occ[dev] > 0 && cache.threads[dev] == threads && cache.smem[dev] == smem) {
         *occ_out = cache.occ[dev];
         return cudaSuccess;
     }
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (!cacheable || smem > cache.attr[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (cacheable) cache.attr[dev] = smem;
+    }
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
     if (e != cudaSuccess) return e;
     if (cacheable) {
-        cache.attr[dev] = true;
+        cache.threads[dev] = threads;
+        cache.smem[dev] = smem;
         cache.occ[dev] = occ;
     }
     *occ_out = occ;

@@ -55,7 +55,8 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int KC = 1024;                  // input channels per work unit
 constexpr int kBlocksPerUnit = KC / 128;  // 128-channel MMA blocks per unit
-constexpr int kActStride = KC / 2 + 64;   // bytes per token row of a staged code chunk
+constexpr int kActWords = KC / 8;         // 8-channel words per token row of a staged chunk
+constexpr int kActStride = kActWords * 8 + 16;  // bytes per token row: (even, odd) word pairs + pad
 constexpr int kMaxSlots = 4;              // code chunks staged per CTA
 constexpr int kMaxTokens = 16;
 constexpr int kMaxChunk = 8192;           // channels rotated per item
@@ -201,23 +202,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
     }
     if (!grid_barrier(p.gbar, p.err, p.limit_ns)) return;
 
-    // ---- phase 2: s_g of the groups this CTA owns; per-token max of |X'| / s_g
+    // ---- phase 2: s_g of the groups this CTA owns; per-token max of |X'| / s_g.
+    // A thread takes one channel of the group and loads it for every token at once.
     for (int g = blockIdx.x; g < NG; g += gridDim.x) {
         float m = 0.0f;
-        for (int e = tid; e < M * G; e += kThreads) {
-            const int t = e / G;
-            const int j = g * G + e % G;
-            m = fmaxf(m, fabsf(__ldcg(p.Xr + (size_t)t * K + __ldg(p.perm + j))));
+        for (int jj = tid; jj < G; jj += kThreads) {
+            const int src = __ldg(p.perm + g * G + jj);
+            float v[kMaxTokens];
+#pragma unroll
+            for (int t = 0; t < kMaxTokens; ++t) v[t] = t < M ? __ldcg(p.Xr + (size_t)t * K + src) : 0.0f;
+#pragma unroll
+            for (int t = 0; t < kMaxTokens; ++t) m = fmaxf(m, fabsf(v[t]));
         }
         float sg = block_max(m, red);
         if (p.unit_scales) sg = 1.0f;
         if (tid == 0) p.s[g] = sg;
         const float sd = sg == 0.0f ? 1.0f : sg;
-        for (int e = tid; e < M * G; e += kThreads) {
-            const int t = e / G;
-            const int j = g * G + e % G;
-            const float x = fabsf(__ldcg(p.Xr + (size_t)t * K + __ldg(p.perm + j)));
-            atomicMax(pam + t, __float_as_uint(__fdiv_rn(x, sd)));
+        for (int jj = tid; jj < G; jj += kThreads) {
+            const int src = __ldg(p.perm + g * G + jj);
+            float v[kMaxTokens];
+#pragma unroll
+            for (int t = 0; t < kMaxTokens; ++t) v[t] = t < M ? __ldcg(p.Xr + (size_t)t * K + src) : 0.0f;
+#pragma unroll
+            for (int t = 0; t < kMaxTokens; ++t)
+                if (t < M) atomicMax(pam + t, __float_as_uint(__fdiv_rn(fabsf(v[t]), sd)));
         }
     }
     __syncthreads();
@@ -243,23 +251,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
             s_sm[g] = sg == 0.0f ? 1.0f : sg;
         }
         __syncthreads();
-        const int TOK = M <= 8 ? 8 : 16;
+        // Staged chunks, as the tensor cores' column operand: per token and 8-channel
+        // word, the codes of the even channels and of the odd ones as int8x4 words of
+        // 16 * code.  A thread takes one word and four tokens (all loads at once).
         const int nslot = u1 > u0 ? (u1 - 1) / p.RT - kc_first + 1 : 0;
-        for (int e = tid; e < nslot * TOK * (KC / 2); e += kThreads) {
-            const int bp = e % (KC / 2);
-            const int t = (e / (KC / 2)) % TOK;
-            const int sl = e / (TOK * (KC / 2));
-            uint32_t byte = 0;
-            if (t < M) {
-                const int j = (kc_first + sl) * KC + 2 * bp;
-                const float* xr = p.Xr + (size_t)t * K;
-                const float sd = s_sm[j / G];
-                const int q0 = code_of(__ldcg(xr + __ldg(p.perm + j)), sd, sc_sm[t]);
-                const int q1 = code_of(__ldcg(xr + __ldg(p.perm + j + 1)), sd, sc_sm[t]);
-                byte = (uint32_t)(q0 & 15) | ((uint32_t)(q1 & 15) << 4);
+        const int TOK = M <= 8 ? 8 : 16;
+        for (int e = tid; e < nslot * kActWords * 4; e += kThreads) {
+            const int wi = e % kActWords;
+            const int tq = (e / kActWords) % 4;
+            const int sl = e / (kActWords * 4);
+            const int j0 = (kc_first + sl) * KC + 8 * wi;
+            const int4 pa = __ldg(reinterpret_cast<const int4*>(p.perm + j0));
+            const int4 pb = __ldg(reinterpret_cast<const int4*>(p.perm + j0 + 4));
+            const int src[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+            const float sd = s_sm[j0 / G];
+            float x[4][8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = tq + 4 * q;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) x[q][c] = t < M ? __ldcg(p.Xr + (size_t)t * K + src[c]) : 0.0f;
             }
-            act[((size_t)sl * kMaxTokens + t) * kActStride + bp] = (uint8_t)byte;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = tq + 4 * q;
+                if (t >= TOK) continue;
+                uint32_t ev = 0, od = 0;
+                if (t < M) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        ev |= ((uint32_t)(code_of(x[q][2 * c], sd, sc_sm[t]) << 4) & 0xF0u) << (8 * c);
+                        od |= ((uint32_t)(code_of(x[q][2 * c + 1], sd, sc_sm[t]) << 4) & 0xF0u) << (8 * c);
+                    }
+                }
+                *reinterpret_cast<uint2*>(act + ((size_t)sl * kMaxTokens + t) * kActStride + 8 * wi) = make_uint2(ev, od);
+            }
         }
+        // packed codes of the owned groups (the layer's qX output)
         for (int g = blockIdx.x; g < NG; g += gridDim.x) {
             for (int e = tid; e < M * (G / 2); e += kThreads) {
                 const int t = e / (G / 2);
@@ -282,6 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
         const bool two = M > 8;
         for (int u = u0 + warp; u < u1; u += kWarps) {
             const int kc = u / p.RT, rt = u % p.RT;
+            {
+                // keep the L2 prefetch kPrefetchUnits units ahead of the loads
+                const int up = u + kPrefetchUnits;
+                if (lane < 16 && up < u1)
+                    prefetch_l2(p.qW + (size_t)((up % p.RT) * 16 + lane) * Kh + (size_t)(up / p.RT) * (KC / 2), KC / 2);
+            }
             const uint8_t* wr = p.qW + (size_t)(rt * 16 + gq) * Kh + (size_t)kc * (KC / 2) + 16 * tq;
             uint4 wa[kBlocksPerUnit], wb[kBlocksPerUnit];
 #pragma unroll
@@ -289,26 +323,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
                 wa[i] = __ldcs(reinterpret_cast<const uint4*>(wr + 64 * i));
                 wb[i] = __ldcs(reinterpret_cast<const uint4*>(wr + (size_t)8 * Kh + 64 * i));
             }
-            const uint8_t* ar = act + ((size_t)(kc - kc_first) * kMaxTokens + gq) * kActStride + 16 * tq;
+            const uint8_t* ar = act + ((size_t)(kc - kc_first) * kMaxTokens + gq) * kActStride + 32 * tq;
             float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
             int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int i = 0; i < kBlocksPerUnit; ++i) {
-                const uint4 x0 = *reinterpret_cast<const uint4*>(ar + 64 * i);
+                // this thread's channels of block i: words 16 i + 4 tq + w, w = 0..3
+                const uint4 b01 = *reinterpret_cast<const uint4*>(ar + 128 * i);
+                const uint4 b23 = *reinterpret_cast<const uint4*>(ar + 128 * i + 16);
+                const uint32_t be[4] = {b01.x, b01.z, b23.x, b23.z}, bo[4] = {b01.y, b01.w, b23.y, b23.w};
                 const uint32_t wA[4] = {wa[i].x, wa[i].y, wa[i].z, wa[i].w};
                 const uint32_t wB[4] = {wb[i].x, wb[i].y, wb[i].z, wb[i].w};
-                const uint32_t xa[4] = {x0.x, x0.y, x0.z, x0.w};
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
-                    mma_s8(d0, nib_even(wA[w]), nib_even(wB[w]), nib_odd(wA[w]), nib_odd(wB[w]), nib_even(xa[w]),
-                           nib_odd(xa[w]));
+                    mma_s8(d0, nib_even(wA[w]), nib_even(wB[w]), nib_odd(wA[w]), nib_odd(wB[w]), be[w], bo[w]);
                 if (two) {
-                    const uint4 x1 = *reinterpret_cast<const uint4*>(ar + (size_t)8 * kActStride + 64 * i);
-                    const uint32_t xb[4] = {x1.x, x1.y, x1.z, x1.w};
+                    const uint8_t* ar1 = ar + (size_t)8 * kActStride;
+                    const uint4 c01 = *reinterpret_cast<const uint4*>(ar1 + 128 * i);
+                    const uint4 c23 = *reinterpret_cast<const uint4*>(ar1 + 128 * i + 16);
+                    const uint32_t ce[4] = {c01.x, c01.z, c23.x, c23.z}, co[4] = {c01.y, c01.w, c23.y, c23.w};
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        mma_s8(d1, nib_even(wA[w]), nib_even(wB[w]), nib_odd(wA[w]), nib_odd(wB[w]), nib_even(xb[w]),
-                               nib_odd(xb[w]));
+                        mma_s8(d1, nib_even(wA[w]), nib_even(wB[w]), nib_odd(wA[w]), nib_odd(wB[w]), ce[w], co[w]);
                 }
                 if ((i + 1) % gpb == 0) {
                     // end of a group: 256 * P_g exactly; promote with s_g

@@ -14,11 +14,14 @@ namespace rrs {
 // its occupancy.  Launch paths call these instead of querying the runtime on
 // every call (the queries cost more host time than a small kernel runs).
 int device_sm_count();
-// Sets the kernel's dynamic shared-memory limit (first call per device) and
-// returns blocks per SM for (threads, smem); `cache` is the kernel's own slot.
+// Raises the kernel's dynamic shared-memory limit to `smem` when needed (it only
+// ever grows, per device) and returns blocks per SM for (threads, smem); `cache`
+// is the kernel's own slot and remembers the last (threads, smem) per device.
 struct KernelSetup {
+    size_t attr[16] = {0};
+    int threads[16] = {0};
+    size_t smem[16] = {0};
     int occ[16] = {0};
-    bool attr[16] = {false};
 };
 cudaError_t kernel_setup(const void* kern, int threads, size_t smem, KernelSetup& cache, int* occ_out);
 

@@ -312,12 +312,11 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     for (int g = threadIdx.x; g < 256; g += blockDim.x) gsm[g] = 0u;
 
     // Gather addresses of this thread's outputs j in [64t, 64t + 64) (one group).
-    // perm is staged through shared memory: 16-byte global loads, four in flight,
-    // and 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each thread's 16
-    // chunk reads below are bank-conflict free.
+    // perm is staged through shared memory (`pst`, K int32): 16-byte global loads,
+    // four in flight, and 16-byte chunk c stored at c ^ ((c >> 4) & 7) so that each
+    // thread's 16 chunk reads below are bank-conflict free.
     uint32_t gaddr[32];
-    {
-        int4* pst = reinterpret_cast<int4*>(rowbufs);
+    auto build_gaddr = [&](int4* pst) {
         const int4* pg = reinterpret_cast<const int4*>(p.perm);
         for (int c0 = 0; c0 < K / 4; c0 += 4 * (int)blockDim.x) {
             int4 v[4];
@@ -340,8 +339,12 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
             gaddr[2 * q] = (uint32_t)swz(v.x) | ((uint32_t)swz(v.y) << 16);
             gaddr[2 * q + 1] = (uint32_t)swz(v.z) | ((uint32_t)swz(v.w) << 16);
         }
-        __syncthreads();   // the row buffers reuse this space
-    }
+        __syncthreads();   // the staging space is reused
+    };
+    // Phase A without kept rows takes its maxima per channel (no gather per row),
+    // and builds the gather addresses afterwards in the staging space.
+    const bool colmax = run_a && !keep;
+    if (!colmax) build_gaddr(reinterpret_cast<int4*>(rowbufs));
     auto gather = [&](float2 (&x)[32]) {
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -356,20 +359,63 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
         // Per row: rotate, reorder (gather), and keep the largest |X'| of this
         // thread's outputs, all of which lie in one group (64 | G).
         float gmx = 0.0f;
-        for (int r = r0; r < p.rows; r += stride, ++it) {
-            advance(r, it);
-            rotate_into_rowbuf(it % nst);
-            float2 x[32];
-            gather(x);
+        if (keep) {
+            // one row per team: rotate into the row buffer (kept for phase B), gather
+            for (int r = r0; r < p.rows; r += stride, ++it) {
+                advance(r, it);
+                rotate_into_rowbuf(it % nst);
+                float2 x[32];
+                gather(x);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) gmx = fmaxf(gmx, fmaxf(fabsf(x[i].x), fabsf(x[i].y)));
-            if (!keep) named_bar(bar_id, T);   // row buffer and staging free for the next row
-        }
-        cp_async_wait<0>();
-        if (!keep && (p.phase & 2)) {
-            // phase B's first rows in flight across the grid barrier
+                for (int i = 0; i < 32; ++i) gmx = fmaxf(gmx, fmaxf(fabsf(x[i].x), fabsf(x[i].y)));
+            }
+            cp_async_wait<0>();
+        } else {
+            // Per row only the rotation; each register keeps the largest |v| of its
+            // channel over this thread's rows (v the unscaled transform: fl(c_n |v|)
+            // is monotone in |v|, so scaling the maximum once gives the same bits).
+            float2 cm[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) cm[i] = make_float2(0.0f, 0.0f);
+            for (int r = r0; r < p.rows; r += stride, ++it) {
+                advance(r, it);
+                const int tl = opaque(t);
+                float2 v[32];
+                rotate_row<L>(v, rowbuf, stage0 + (size_t)(it % nst) * K, tl, T, bar_id);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    cm[i].x = fmaxf(cm[i].x, fabsf(v[i].x));
+                    cm[i].y = fmaxf(cm[i].y, fabsf(v[i].y));
+                }
+                named_bar(bar_id, T);   // row buffer and staging free for the next row
+            }
+            cp_async_wait<0>();
             __syncthreads();
-            prologue();
+            // channel maxima in natural order (swizzled) in every team's buffer, then
+            // the CTA's maxima in team 0's buffer (same swizzle: combine position-wise)
+            store_natural<L>(cm, rowbuf, opaque(t), T);
+            __syncthreads();
+            if (R > 1) {
+                for (int c = threadIdx.x; c < K; c += blockDim.x) {
+                    float m = rowbufs[c];
+                    for (int q = 1; q < R; ++q) m = fmaxf(m, rowbufs[(size_t)q * K + c]);
+                    rowbufs[c] = m;
+                }
+                __syncthreads();
+            }
+            build_gaddr(reinterpret_cast<int4*>(stages0));
+            if (team == 0) {
+                float2 x[32];
+                gather(x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) gmx = fmaxf(gmx, fmaxf(x[i].x, x[i].y));
+                gmx = __fmul_rn(gmx, p.c_n);
+            }
+            if (p.phase & 2) {
+                // phase B's first rows in flight across the grid barrier
+                __syncthreads();
+                prologue();
+            }
         }
         // threads of one group are consecutive (G / 64 of them): shuffle-reduce
         // within aligned power-of-two segments, one shared atomic per segment

@@ -267,6 +267,12 @@ def run_ours(args):
                                     for j in range(len(state))],
               "weights": "INT4 codes packed two per byte (N*K/2 bytes); int8 tensor-core GEMM"}
 
+    # ---- the gated MLP block at LLaMA-3-8B sizes on the same path (timed apart from the step)
+    mlp = None if args.no_mlp else mlp_block_times(rrs, wl, dev, stream, args.warmup, max(3, min(K, 200)), pg)
+
+    # ---- decode (70B q/o, one token; the single-launch layer) and the INT4 KV cache
+    extra = {} if args.no_mlp else extra_rows(rrs, wl, dev, pg)
+
     # ---- end to end through the C ABI with host buffers (pinned), copies timed.
     e2e = None
     if not args.no_e2e:
@@ -322,6 +328,8 @@ def run_ours(args):
         "gemm": {"ms_per_layer": [round(x, 5) for x in gemm_ms], "TOPS": round(gemm_tops, 1)},
         "e2e": e2e,
         "packed_weights": packed,
+        "mlp_block": mlp,
+        **extra,
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
     }
@@ -332,6 +340,114 @@ def run_ours(args):
         pg.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def extra_rows(rrs, wl, dev, pg):
+    """Two more rows measured in the same run, apart from the step: the single-launch
+    layer for one decode token (70B q/o, weights rotated past L2) and the INT4 KV cache
+    of a batch (quantise and dequantise), each against the HBM peak."""
+    _, hbm_peak, _ = peaks()
+    L = wl.LAYERS["llama3_70b_qo_decode_m1"]
+    dec = decode_entry(rrs, wl, dev, L, wl.make_activations(L).to(dev), wl.make_weights(L).to(dev), hbm_peak)
+    torch.cuda.empty_cache()
+    # KV cache of LLaMA-3-70B (8 KV heads of 128) for 16 sequences of 4096 tokens
+    T, H, D = 65536, 8, 128
+    g = torch.Generator().manual_seed(404)
+    kv = (torch.randn(T, H, D, generator=g) * 2.0)
+    kv[:, :, 5] *= 40.0
+    kv = kv.to(torch.float16).to(dev)
+    q = torch.empty((T, H, D // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((T, H), dtype=torch.float32, device=dev)
+    out = torch.empty_like(kv)
+    tq = _time_ms(lambda: rrs.kv_quant(kv, q=q, scale=sc), 10)
+    td = _time_ms(lambda: rrs.kv_dequant(q, sc, out=out), 10)
+    n = T * H * D
+    bq = 2 * n + n // 2 + 4 * T * H
+    bd = n // 2 + 4 * T * H + 2 * n
+    tq, td = max_over_ranks(tq, pg, dev), max_over_ranks(td, pg, dev)
+    kvr = {"T": T, "H": H, "D": D, "quant_us": round(tq * 1e3, 2), "dequant_us": round(td * 1e3, 2),
+           "quant_GBps": round(bq / (tq * 1e-3) / 1e9, 1), "dequant_GBps": round(bd / (td * 1e-3) / 1e9, 1),
+           "quant_frac_hbm": round(bq / (tq * 1e-3) / 1e9 / hbm_peak, 4),
+           "dequant_frac_hbm": round(bd / (td * 1e-3) / 1e9 / hbm_peak, 4),
+           "bytes": "quantise: fp16 in, packed codes + fp32 scales out; dequantise: the reverse"}
+    del kv, q, sc, out
+    torch.cuda.empty_cache()
+    return {"decode": dec, "kv_cache": kvr}
+
+
+def mlp_block_times(rrs, wl, dev, stream, warmup, iters, pg):
+    """The gated MLP block of LLaMA-3-8B (M = 2048 tokens, K = 4096, F = 14336, G = 128):
+    gate/up RRS linear on the fp8 path with SiLU * up fused into its GEMM epilogue
+    (interleaved gate/up weight rows), then the down RRS linear (block-diagonal rotation,
+    7 blocks of 2048) on H.  Four launches per block; CUDA events around each."""
+    M, K, F, G = 2048, 4096, 14336, 128
+    Lgu = wl.Layer("llama3_8b_mlp_gateup", M, K, 2 * F, G, 4096, seed=501)
+    Lu = wl.Layer("llama3_8b_mlp_up", M, K, F, G, 4096, seed=503)
+    Ld = wl.Layer("llama3_8b_mlp_down", M, F, K, G, 2048, seed=502)
+    W = rrs.interleave_gate_up(wl.make_weights(Lgu, N=F), wl.make_weights(Lu)).to(dev)
+    perm_gu = rrs.calibrate_perm(wl.make_activations(Lgu, sample=1, M=512).to(dev), Lgu.had_block)
+    qW, sw_gu = rrs.prepare_weights(W, perm_gu, Lgu.had_block)
+    qW_gu = rrs.expand_weights(qW)
+    del W, qW
+    xs = [wl.make_activations(Lgu, sample=2 + i).to(dev) for i in range(2)]
+    flags = rrs.W_EXPANDED
+    qX = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty(K // G, dtype=torch.float32, device=dev)
+    st = torch.empty(M, dtype=torch.float32, device=dev)
+    H = torch.empty((M, F), dtype=torch.float16, device=dev)
+    ws = rrs.make_workspace(M, 2 * F, K, G, Lgu.had_block, flags, device=dev)
+    # calibration of the down projection's reorder on the H of a calibration draw
+    rrs.linear(wl.make_activations(Lgu, sample=1).to(dev), qW_gu, sw_gu, perm_gu, G, Lgu.had_block,
+               flags=flags | rrs.Y_SILU_MUL, Y=H, qX=qX, s=s, scale_t=st, ws=ws)
+    perm_d = rrs.calibrate_perm(H[:512], Ld.had_block)
+    Wd = wl.make_weights(Ld).to(dev)
+    qWd, sw_d = rrs.prepare_weights(Wd, perm_d, Ld.had_block)
+    qW_d = rrs.expand_weights(qWd)
+    del Wd, qWd
+    qXd = torch.empty((M, F // 2), dtype=torch.uint8, device=dev)
+    sd = torch.empty(F // G, dtype=torch.float32, device=dev)
+    std = torch.empty(M, dtype=torch.float32, device=dev)
+    Yd = torch.empty((M, K), dtype=torch.float32, device=dev)
+    wsd = rrs.make_workspace(M, K, F, G, Ld.had_block, flags, device=dev)
+
+    def block(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rrs.smooth_quant(xs[i % 2], perm_gu, G, Lgu.had_block, flags=flags, qX=qX, s=s, scale_t=st, ws=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        rrs.w4a4_gemm(qX, s, st, qW_gu, sw_gu, G, Y=H, ws=ws, flags=rrs.WS_HOLDS_A8 | flags | rrs.Y_SILU_MUL)
+        if ev is not None:
+            ev[2].record(stream)
+        rrs.smooth_quant(H, perm_d, G, Ld.had_block, flags=flags, qX=qXd, s=sd, scale_t=std, ws=wsd)
+        if ev is not None:
+            ev[3].record(stream)
+        rrs.w4a4_gemm(qXd, sd, std, qW_d, sw_d, G, Y=Yd, ws=wsd, flags=rrs.WS_HOLDS_A8 | flags)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for i in range(warmup):
+        block(i)
+    rrs.check_workspace(ws)
+    rrs.check_workspace(wsd)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(iters)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    for i in range(iters):
+        block(i, evs[i])
+    torch.cuda.synchronize()
+    rrs.check_workspace(ws)
+    rrs.check_workspace(wsd)
+    stages = ["gateup_prep", "gateup_gemm_silu_mul", "down_prep", "down_gemm"]
+    us = {nm: sum(e[k].elapsed_time(e[k + 1]) for e in evs) / iters * 1e3 for k, nm in enumerate(stages)}
+    total = sum(e[0].elapsed_time(e[4]) for e in evs) / iters * 1e3
+    total = max_over_ranks(total, pg, dev)
+    ops = 2 * M * (2 * F) * K + 2 * M * K * F
+    return {"M": M, "K": K, "F": F, "G": G, "down_hadamard": "7 x 2048", "iters": iters,
+            "us": {k: round(v, 2) for k, v in us.items()}, "us_total": round(total, 2),
+            "TOPS": round(ops / (total * 1e-6) / 1e12, 1), "launches": 4,
+            "path": "fp8 (e4m3) MMA; SiLU * up fused into the gate/up GEMM epilogue (H fp16 written once)"}
 
 
 def _oracle_sample(layers, rows_per_layer, cols_per_layer=None, seed=0):
@@ -640,6 +756,7 @@ def main():
     ap.add_argument("--workload", default="", help="comma-separated layer names (default: headline shapes)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mlp", action="store_true", help="skip the MLP-block, decode and KV-cache rows")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--report", action="store_true",
                     help="print the other configurations (group sweep, 8B down, 70B, decode) instead")

@@ -154,3 +154,47 @@ def test_silu_mul_flag_needs_the_fp8_path(rrs):
         rrs.w4a4_gemm(qX, s, torch.ones(4, device=DEV), qW, torch.ones(8, device=DEV), 128, flags=rrs.Y_SILU_MUL)
     assert e.value.status_name == "RRS_ERR_UNSUPPORTED"
 
+
+
+def test_fused_mlp_block_at_llama3_8b_sizes(rrs):
+    """The product's MLP block at LLaMA-3-8B sizes (M = 2048, K = 4096, F = 14336; the
+    down projection's rotation block-diagonal with 7 blocks of 2048): gate/up RRS linear
+    on the fp8 path with SiLU * up fused into its epilogue (interleaved weight rows),
+    then the down RRS linear on H.  Stage by stage against the oracle: every code and
+    scale of both linears bit for bit over all tokens (the down projection fed the GPU's
+    own H), sampled rows of the gate/up output and of Y within the tolerance, and the
+    fused H equal bit for bit to SiLU * up of the unfused fp32 output."""
+    M, K, F, G = 2048, 4096, 14336, 128
+    up = wl.Layer("llama3_8b_mlp_gateup", M, K, 2 * F, G, 4096, seed=501)
+    down = wl.Layer("llama3_8b_mlp_down", M, F, K, G, 2048, seed=502)
+    X = wl.make_activations(up)
+    Wgu = rrs.interleave_gate_up(wl.make_weights(up, N=F), wl.make_weights(wl.Layer("u", M, K, F, G, 4096, seed=503)))
+    perm_gu = wl.random_perm(K, 21)
+    Xd, pgu = X.to(DEV), perm_gu.to(DEV)
+    qW, sw = rrs.prepare_weights(Wgu.to(DEV), pgu, up.had_block)
+    qW8 = rrs.expand_weights(qW)
+    qX = torch.empty((M, K // 2), dtype=torch.uint8, device=DEV)
+    s = torch.empty(K // G, dtype=torch.float32, device=DEV)
+    st = torch.empty(M, dtype=torch.float32, device=DEV)
+    H = rrs.linear(Xd, qW8, sw, pgu, G, up.had_block, flags=rrs.W_EXPANDED | rrs.Y_SILU_MUL, qX=qX, s=s, scale_t=st)
+    GU = rrs.linear(Xd, qW8, sw, pgu, G, up.had_block, flags=rrs.W_EXPANDED)
+    torch.cuda.synchronize()
+    assert H.shape == (M, F) and H.dtype == torch.float16
+    Href = rrs.silu_mul(torch.cat([GU[:, 0::2], GU[:, 1::2]], dim=1).contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(H.view(torch.int16), Href.view(torch.int16))
+    _, oqX, os_, ost = oracle.smooth_quant(X, G, up.had_block, perm_gu.numpy())
+    for got, want, what in ((qX, oqX, "qX"), (s, os_, "s"), (st, ost, "scale_t")):
+        assert np.array_equal(got.cpu().numpy().view(np.uint8), np.asarray(want).view(np.uint8)), what
+    _, oqW, osw = oracle.prepare_weights(Wgu, up.had_block, perm_gu.numpy())
+    assert np.array_equal(qW.cpu().numpy(), oqW)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), osw.view(np.uint32))
+    rows = [0, 1, 777, 1500, M - 1] + [int(r) for r in np.argsort(ost)[-3:]]
+    Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
+    ok = oracle.y_tolerance_ok(GU.cpu().numpy()[rows], Yo, B)
+    assert ok.all(), f"gate/up: {np.count_nonzero(~ok)} of {ok.size} outside tolerance"
+    del GU, Href, qW8
+    # the down projection on the GPU's H, with the calibrated reorder of its channels
+    Wd = wl.make_weights(down)
+    perm_d = torch.from_numpy(oracle.calibrate_perm(H[:256].cpu(), down.had_block))
+    _linear_checked(rrs, H, Wd, perm_d, G, down.had_block, rows=rows)

@@ -506,3 +506,22 @@ def test_llama3_70b_prefill_layers(rrs, name):
     perm = wl.random_perm(L.K, 5)
     _, _, _, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
     run_layer(rrs, X, W, perm, L.G, L.had_block, rows=_sample_rows(L.M, ost, k=8))
+
+
+def test_one_hadamard_size_at_two_row_lengths_in_sequence(rrs):
+    """The activation kernel for one Hadamard size serves row lengths that need
+    different shared memory (K = 14336 with 7 blocks of 2048, then K = 2048 with 8
+    rows per CTA): the second launch must get its own shared-memory limit."""
+    L = wl.LAYERS["llama3_8b_down"]
+    X1 = wl.make_activations(L, M=64)
+    p1 = wl.random_perm(L.K, 31)
+    rrs.smooth_quant(X1.to(DEV), p1.to(DEV), L.G, L.had_block)
+    g = torch.Generator().manual_seed(32)
+    X2 = (torch.randn(256, 2048, generator=g) * 2).to(torch.float16)
+    p2 = wl.random_perm(2048, 32)
+    qX, s, st = rrs.smooth_quant(X2.to(DEV), p2.to(DEV), 128, 2048)
+    torch.cuda.synchronize()
+    _, oqX, os_, ost = oracle.smooth_quant(X2, 128, 2048, p2.numpy())
+    assert_bits_equal(s, os_, "s")
+    assert_bits_equal(st, ost, "scale_t")
+    assert_bits_equal(qX, oqX, "qX")
