@@ -222,6 +222,24 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t* err, uint
     return ok_s != 0;
 }
 
+// Division a / b for b > 0 by Markstein's method (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990): with y = RN(1/b) and q0 = RN(a*y), the residual
+// r = a - b*q0 is exact (one fma) and RN(q0 + r*y) is the correctly rounded
+// quotient RN(a/b), barring underflow/overflow of the intermediates, which the
+// value ranges here exclude (|a| <= b, |a| >= 2^-40 or a == 0).  It is checked
+// against the IEEE division in the GPU tests.
+__device__ __forceinline__ float2 div_markstein(float2 a, float2 nb, float2 y) {
+    const float2 q0 = __fmul2_rn(a, y);
+    const float2 r = __ffma2_rn(q0, nb, a);
+    return __ffma2_rn(r, y, q0);
+}
+__device__ __forceinline__ float div_markstein(float a, float nb, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float r = __fmaf_rn(q0, nb, a);
+    return __fmaf_rn(r, y, q0);
+}
+
 // The gated-MLP activation of one output: silu(g) * u with silu(g) = g / (1 +
 // exp(-g)) in fp32, saturated to +-65504 (the fp16 range the next layer's
 // activation path takes); the caller rounds it to fp16.  One definition for the

@@ -115,18 +115,6 @@ __device__ __forceinline__ void rstore(const float2 (&v)[32], float* buf, int t,
 
 
 // ---------------------------------------------------------------------------
-// Division a / b for b > 0 by Markstein's method (P. Markstein, "Computation of
-// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
-// Dev. 34(1), 1990): with y = RN(1/b) and q0 = RN(a*y), the residual
-// r = a - b*q0 is exact (one fma) and RN(q0 + r*y) is the correctly rounded
-// quotient RN(a/b), barring underflow/overflow of the intermediates, which the
-// value ranges here exclude (|a| <= b, |a| >= 2^-40 or a == 0).  It is checked
-// against the IEEE division in the GPU tests.
-__device__ __forceinline__ float2 div_markstein(float2 a, float2 nb, float2 y) {
-    const float2 q0 = __fmul2_rn(a, y);
-    const float2 r = __ffma2_rn(q0, nb, a);
-    return __ffma2_rn(r, y, q0);
-}
 
 
 // Gathers byte 0 of four words into one word: result byte i = byte 0 of w_i.

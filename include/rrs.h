@@ -120,7 +120,10 @@ typedef enum {
  * K/128 floats per CTA of the activation kernel (at most 1024 rows).  For
  * M <= 16 and N > 0 the space after the operand is at least 16*M*N*4 bytes: the
  * packed-weight GEMM then splits k across CTAs and keeps its partial sums there
- * (the table is dead by then).  rrs_w4a4_gemm alone needs only the first two
+ * (the table is dead by then); and the space after the header also holds the
+ * single-launch layer of rrs_linear (rotated rows M*K*4 bytes, a per-CTA table of
+ * 16 token maxima for up to 1024 CTAs, N/16 tile counters, and K/1024 chunk sums
+ * of M*N*4 bytes each, every part 256-byte aligned).  rrs_w4a4_gemm alone needs only the first two
  * parts; given less room it simply does not split.  N = 0 sizes a workspace for
  * the activation calls alone.  One workspace must not be used by two calls in
  * flight at the same time.  A call that times out (RRS_ERR_TIMEOUT) may leave
@@ -183,7 +186,14 @@ rrs_status rrs_w4a4_gemm(const uint8_t *qX, const float *s, const float *scale_t
                          size_t ws_bytes, unsigned flags, rrs_stream_t stream);
 
 /* rrs_smooth_quant followed by rrs_w4a4_gemm on one stream, no host sync.
- * qX, s and scale_t are caller-provided intermediate buffers. */
+ * qX, s and scale_t are caller-provided intermediate buffers (written as by
+ * rrs_smooth_quant).  For M <= 16 tokens with packed weights (no
+ * RRS_W_EXPANDED, no RRS_Y_SILU_MUL), N % 16 == 0, K % 1024 == 0, G dividing
+ * 1024 and a workspace of rrs_workspace_size(M, N, ...) bytes, the whole layer
+ * runs as one cooperative kernel instead: the same codes, s and scale_t bit for
+ * bit, and Y differing only in the order of its fp32 sums over 1024-channel
+ * chunks (summed in chunk order).  Other shapes, or a smaller workspace, take the
+ * two launches. */
 rrs_status rrs_linear(const void *X, const uint8_t *qW, const float *scale_w, const int32_t *perm,
                       int M, int N, int K, int G, int had_block, uint8_t *qX, float *s,
                       float *scale_t, float *Y, void *ws, size_t ws_bytes, unsigned flags,
