@@ -8,7 +8,7 @@ synthetic workloads.  Build the library with
 from . import workloads  # noqa: F401  (no CUDA needed)
 
 _API = (
-    "NO_ROTATE", "FORCE_UNIT_SCALES", "WS_HOLDS_A8", "W_EXPANDED", "Y_BF16", "Y_SILU_MUL", "interleave_gate_up", "RRSError", "lib", "workspace_size", "make_workspace",
+    "NO_ROTATE", "FORCE_UNIT_SCALES", "WS_HOLDS_A8", "W_EXPANDED", "Y_BF16", "Y_SILU_MUL", "ONE_LAUNCH", "interleave_gate_up", "RRSError", "lib", "workspace_size", "make_workspace",
     "prepare_weights", "smooth_quant", "group_max", "smooth_quant_scaled", "w4a4_gemm", "linear", "linear_from_host",
     "w4a4_gemm_debug_partials", "channel_absmax", "perm_from_channel_max", "calibrate_perm",
     "check_workspace", "check_perm", "debug_wait_timeout", "debug_divide", "expand_weights", "silu_mul", "kv_quant", "kv_dequant", "LIB_PATH",

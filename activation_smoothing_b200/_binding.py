@@ -23,6 +23,7 @@ WS_HOLDS_A8 = 4
 W_EXPANDED = 8
 Y_BF16 = 16
 Y_SILU_MUL = 32
+ONE_LAUNCH = 64
 
 _STATUS = {
     0: "RRS_OK",

@@ -486,7 +486,8 @@ rrs_status rrs_linear(const void* X, const uint8_t* qW, const float* scale_w, co
         if (r != RRS_OK) return r;
         r = check_ws(ws, ws_bytes, ws_bytes_full(M, K, n));
         if (r != RRS_OK) return r;
-        if (ws_bytes >= kHeaderBytes + rrs::decode_ws_bytes(M, N, K) && rrs::decode_supported(M, N, K, G, n)) {
+        if (ws_bytes >= kHeaderBytes + rrs::decode_ws_bytes(M, N, K) && rrs::decode_supported(M, N, K, G, n) &&
+            ((flags & RRS_ONE_LAUNCH) || rrs::decode_preferred(M, N, K))) {
             rrs::DecodeLaunch dl{};
             dl.X = X;
             dl.perm = perm;

@@ -32,9 +32,10 @@
 //            sign extension needed), and multiplies on the tensor cores with
 //            mma.sync m16n8k32 (weights as the 16-row operand, tokens as the
 //            8 columns).  Each group's exact sum 256 * P_g is shifted back and
-//            promoted, acc += s_g * P_g, in group order.  A unit's sums go to
-//            the workspace; the last unit of an output tile to finish adds the
-//            chunks in order and applies scale_t * scale_w.
+//            promoted, acc += s_g * P_g, in group order; a unit's sums go to
+//            the workspace;                                 -- grid barrier
+//   phase 4  every thread of the grid takes outputs: the chunk sums added in
+//            chunk order, times scale_t * scale_w.
 //
 // All integer results (codes, s, scale_t) are the same bits the two-launch
 // path gives; Y differs from it only in the order of the fp32 sums over chunks.
@@ -97,7 +98,6 @@ struct Args {
     int ybf16;
     float* Xr;      // [M, K] rotated activations
     float* gtab;    // [M, K / L, NG] largest |X_rot| of each rotation item per group
-    int* cnt;       // [N / 16] finished units per output tile
     float* part;    // [K / KC, M, N] per-chunk sums
     int L;          // channels per rotation item: max(n, 1024)
     int RT, KCN, U; // output tiles, chunks, units
@@ -226,8 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
     const int u1 = (int)((long long)(blockIdx.x + 1) * p.U / gridDim.x);
     const int kc_first = u0 / p.RT;
 
-    // ---- phase 0: start the weight stream (L2 prefetch), clear the tile counters,
-    // and invert the reorder: channel perm[j] of the rotated row lies in group j / G
+    // ---- phase 0: start the weight stream (L2 prefetch) and invert the reorder: channel perm[j] of the rotated row lies in group j / G
     {
         const int npf = min(u1 - u0, kPrefetchUnits);
         for (int e = tid; e < npf * 16; e += kThreads) {
@@ -235,7 +234,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
             const int row = (u % p.RT) * 16 + (e % 16);
             prefetch_l2(p.qW + (size_t)row * Kh + (size_t)(u / p.RT) * (KC / 2), KC / 2);
         }
-        for (int i = blockIdx.x * kThreads + tid; i < p.RT; i += gridDim.x * kThreads) p.cnt[i] = 0;
         const int4* p4 = reinterpret_cast<const int4*>(p.perm);
         for (int b = tid; b < K / 4; b += kThreads * 8) {
             int4 v[8];
@@ -533,37 +531,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
                 if (t0 < M) pc[(size_t)t0 * N + row] = acc0[r];
                 if (two && t0 + 8 < M) pc[(size_t)(t0 + 8) * N + row] = acc1[r];
             }
-            __threadfence();
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) last = atomicAdd(p.cnt + rt, 1) == p.KCN - 1;
-            last = __shfl_sync(0xFFFFFFFFu, last, 0);
-            if (last) {
-                __threadfence();
-                const size_t cs = (size_t)M * N;   // stride between chunks
-                for (int e = lane; e < 16 * M; e += 32) {
-                    const int row = rt * 16 + (e & 15);
-                    const int t = e >> 4;
-                    const float* pp = p.part + (size_t)t * N + row;
-                    // the chunks' sums in chunk order, eight loads in flight at a time
-                    float a = __ldcg(pp);
-                    int c = 1;
-                    for (; c + 8 <= p.KCN; c += 8) {
-                        float w[8];
+        }
+    }
+    // every unit's sums are in the workspace
+    if (!grid_barrier(p.gbar, p.err, p.limit_ns)) return;
+
+    // ---- phase 4: Y = (sum of the chunk sums, in chunk order) * scale_t * scale_w,
+    // one output per thread across the grid, eight chunk loads in flight at a time
+    {
+        const size_t cs = (size_t)M * N;   // stride between chunks
+        for (size_t e = (size_t)blockIdx.x * kThreads + tid; e < cs; e += (size_t)gridDim.x * kThreads) {
+            const int t = (int)(e / N);
+            const int row = (int)(e % N);
+            const float* pp = p.part + e;
+            float a = __ldcg(pp);
+            int c = 1;
+            for (; c + 8 <= p.KCN; c += 8) {
+                float w[8];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) w[q] = __ldcg(pp + (size_t)(c + q) * cs);
+                for (int q = 0; q < 8; ++q) w[q] = __ldcg(pp + (size_t)(c + q) * cs);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) a = __fadd_rn(a, w[q]);
-                    }
-                    for (; c < p.KCN; ++c) a = __fadd_rn(a, __ldcg(pp + (size_t)c * cs));
-                    const float y = __fmul_rn(__fmul_rn(a, sc_sm[t]), __ldg(p.scale_w + row));
-                    if (p.ybf16)
-                        reinterpret_cast<__nv_bfloat16*>(p.Y)[(size_t)t * N + row] = __float2bfloat16_rn(y);
-                    else
-                        reinterpret_cast<float*>(p.Y)[(size_t)t * N + row] = y;
-                }
-                if (lane == 0) p.cnt[rt] = 0;
+                for (int q = 0; q < 8; ++q) a = __fadd_rn(a, w[q]);
             }
+            for (; c < p.KCN; ++c) a = __fadd_rn(a, __ldcg(pp + (size_t)c * cs));
+            const float y = __fmul_rn(__fmul_rn(a, sc_sm[t]), __ldg(p.scale_w + row));
+            if (p.ybf16)
+                reinterpret_cast<__nv_bfloat16*>(p.Y)[e] = __float2bfloat16_rn(y);
+            else
+                reinterpret_cast<float*>(p.Y)[e] = y;
         }
     }
 }
@@ -591,13 +586,16 @@ bool decode_supported(int M, int N, int K, int G, int n) {
     return true;
 }
 
-// Workspace bytes after the 256-byte header: X_rot, the per-item group maxima,
-// the tile counters and the per-chunk sums, each 256-byte aligned.
+// Where the single launch is the faster form (measured on the 70B decode layers):
+// few tokens, or a weight stream large enough to hide the activation phases.
+bool decode_preferred(int M, int N, int K) { return M <= 4 || (long long)N * K >= (1LL << 27); }
+
+// Workspace bytes after the 256-byte header: X_rot, the per-item group maxima
+// and the per-chunk sums, each 256-byte aligned.
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 static size_t gtab_bytes(int M, int K) { return (size_t)M * (K / dec::kMinChunk) * (K / 128) * 4; }
 size_t decode_ws_bytes(int M, int N, int K) {
-    return al256((size_t)M * K * 4) + al256(gtab_bytes(M, K)) + al256((size_t)(N / 16) * 4) +
-           al256((size_t)(K / dec::KC) * M * N * 4);
+    return al256((size_t)M * K * 4) + al256(gtab_bytes(M, K)) + al256((size_t)(K / dec::KC) * M * N * 4);
 }
 
 cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t st) {
@@ -630,8 +628,6 @@ cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t st) {
     w += al256((size_t)dl.M * dl.K * 4);
     a.gtab = reinterpret_cast<float*>(w);
     w += al256(gtab_bytes(dl.M, dl.K));
-    a.cnt = reinterpret_cast<int*>(w);
-    w += al256((size_t)(dl.N / 16) * 4);
     a.part = reinterpret_cast<float*>(w);
     a.L = dl.n > kMinChunk ? dl.n : kMinChunk;
     a.RT = dl.N / 16;

@@ -110,6 +110,7 @@ struct DecodeLaunch {
     uint32_t* err;
 };
 bool decode_supported(int M, int N, int K, int G, int n);
+bool decode_preferred(int M, int N, int K);
 size_t decode_ws_bytes(int M, int N, int K);
 cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t stream);
 

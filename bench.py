@@ -660,8 +660,8 @@ def run_report(args):
 
 
 def decode_entry(rrs, wl, dev, L, X, W, hbm_peak, iters=24):
-    """A decode layer (M <= 16): rrs_linear (one launch) against the two launches
-    (activation kernel, then the GEMM).  Each timed call reads its own copy of the
+    """A decode layer (M <= 16): rrs_linear as it chooses, its single launch forced
+    (RRS_ONE_LAUNCH), and the two launches (activation kernel, then the GEMM).  Each timed call reads its own copy of the
     packed weights, enough copies that they exceed L2, so the weight stream comes
     from HBM as it would in a model's layer sequence."""
     n = L.had_block
@@ -681,7 +681,9 @@ def decode_entry(rrs, wl, dev, L, X, W, hbm_peak, iters=24):
         k[0] = (k[0] + 1) % copies
         return qWs[k[0]]
 
-    one = _time_ms(lambda: rrs.linear(X, nxt(), sw, perm, L.G, n, Y=Y, qX=qX, s=s, scale_t=st, ws=ws), iters)
+    one = _time_ms(lambda: rrs.linear(X, nxt(), sw, perm, L.G, n, flags=rrs.ONE_LAUNCH, Y=Y, qX=qX, s=s,
+                                      scale_t=st, ws=ws), iters)
+    dflt = _time_ms(lambda: rrs.linear(X, nxt(), sw, perm, L.G, n, Y=Y, qX=qX, s=s, scale_t=st, ws=ws), iters)
     rrs.check_workspace(ws)
 
     def two_launches():
@@ -693,6 +695,7 @@ def decode_entry(rrs, wl, dev, L, X, W, hbm_peak, iters=24):
     rrs.check_workspace(ws)
     gbps = wbytes / (one * 1e-3) / 1e9
     return {"layer": L.name, "M": L.M, "K": L.K, "N": L.N, "G": L.G, "n": n,
+            "rrs_linear_us": round(dflt * 1e3, 2),
             "single_launch_us": round(one * 1e3, 2), "two_launches_us": round(two * 1e3, 2),
             "prep_us": round(prep * 1e3, 2), "weight_copies_rotated": copies,
             "single_launch_weight_GBps": round(gbps, 1),

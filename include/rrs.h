@@ -110,6 +110,12 @@ typedef enum {
                                     from the fp32 Y it would have stored, with rrs_silu_mul's
                                     arithmetic (same bits).  Pass H cast to float *.  Saves
                                     writing and reading the fp32 gate/up output. */
+#define RRS_ONE_LAUNCH 64u       /* rrs_linear, rrs_linear_from_host: for M <= 16 with packed
+                                    weights, always take the single-launch layer where the
+                                    shape allows it.  Without it the single launch is taken
+                                    only where it is the faster of the two forms: M <= 4, or
+                                    N * K >= 2^27 (the weight stream then outweighs the
+                                    fixed cost of the in-kernel activation phases). */
 
 /* Bytes of workspace the calls below need for this problem.  Layout: a
  * 256-byte header (zero-fill it once before first use: it holds the kernels'
@@ -121,9 +127,9 @@ typedef enum {
  * M <= 16 and N > 0 the space after the operand is at least 16*M*N*4 bytes: the
  * packed-weight GEMM then splits k across CTAs and keeps its partial sums there
  * (the table is dead by then); and the space after the header also holds the
- * single-launch layer of rrs_linear (rotated rows M*K*4 bytes, a per-CTA table of
- * 16 token maxima for up to 1024 CTAs, N/16 tile counters, and K/1024 chunk sums
- * of M*N*4 bytes each, every part 256-byte aligned).  rrs_w4a4_gemm alone needs only the first two
+ * single-launch layer of rrs_linear (rotated rows M*K*4 bytes, a table of group
+ * maxima of M*(K/1024)*(K/128) floats, and K/1024 chunk sums of M*N*4 bytes each,
+ * every part 256-byte aligned).  rrs_w4a4_gemm alone needs only the first two
  * parts; given less room it simply does not split.  N = 0 sizes a workspace for
  * the activation calls alone.  One workspace must not be used by two calls in
  * flight at the same time.  A call that times out (RRS_ERR_TIMEOUT) may leave
@@ -190,7 +196,8 @@ rrs_status rrs_w4a4_gemm(const uint8_t *qX, const float *s, const float *scale_t
  * rrs_smooth_quant).  For M <= 16 tokens with packed weights (no
  * RRS_W_EXPANDED, no RRS_Y_SILU_MUL), N % 16 == 0, K % 1024 == 0, G dividing
  * 1024 and a workspace of rrs_workspace_size(M, N, ...) bytes, the whole layer
- * runs as one cooperative kernel instead: the same codes, s and scale_t bit for
+ * can run as one cooperative kernel instead (where it is faster, or always
+ * under RRS_ONE_LAUNCH): the same codes, s and scale_t bit for
  * bit, and Y differing only in the order of its fp32 sums over 1024-channel
  * chunks (summed in chunk order).  Other shapes, or a smaller workspace, take the
  * two launches. */
