@@ -479,22 +479,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 //   tempty[b] even CTA only: 16 arrivals, the epilogue warps of both CTAs
 // No load uses cluster multicast; the only multicast is tcgen05.commit's.
 namespace pair {
-constexpr int BN = 256;                       // tile columns (both CTAs)
-constexpr int BNH = 128;                      // weight rows loaded per CTA
-constexpr int KPS = 2;                        // k-blocks per stage: one 3-D copy per operand carries both
-constexpr int A_TILE = BM * BK;               // 16 KB: one k-block of activation rows
-constexpr int B_TILE = BNH * BK;              // 16 KB: one k-block of weight rows
-constexpr int A_STAGE = KPS * A_TILE;
-constexpr int B_STAGE = KPS * B_TILE;
-constexpr int STAGE = A_STAGE + B_STAGE;      // 64 KB per CTA
-constexpr int NST = 3;
-constexpr int NBUF = 2;                       // TMEM buffers of 256 columns
-constexpr int OFF_B = NST * A_STAGE;
-constexpr int OFF_BAR = OFF_B + NST * B_STAGE;
-constexpr int OFF_S = OFF_BAR + 1024;
-constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
-static_assert(SMEM <= 227 * 1024, "shared memory budget");
-static_assert(2 * NST <= 32, "two lanes per stage");
+// Tile shape of the pair: 256 rows x PBN columns (PBN = 256, or 128 for narrow N).
+template <int PBN>
+struct PCfg {
+    static constexpr int BN = PBN;                      // tile columns (both CTAs)
+    static constexpr int BNH = PBN / 2;                 // weight rows loaded per CTA
+    static constexpr int KPS = 2;                       // k-blocks per stage: one 3-D copy per operand carries both
+    static constexpr int A_TILE = BM * BK;              // 16 KB: one k-block of activation rows
+    static constexpr int B_TILE = BNH * BK;             // one k-block of weight rows
+    static constexpr int A_STAGE = KPS * A_TILE;
+    static constexpr int B_STAGE = KPS * B_TILE;
+    static constexpr int STAGE = A_STAGE + B_STAGE;     // 64 KB (PBN 256) or 48 KB per CTA
+    static constexpr int NST = PBN == 256 ? 3 : 4;
+    static constexpr int NBUF = 512 / PBN;              // TMEM accumulator buffers of PBN columns
+    static constexpr int OFF_B = NST * A_STAGE;
+    static constexpr int OFF_BAR = OFF_B + NST * B_STAGE;
+    static constexpr int OFF_S = OFF_BAR + 1024;
+    static constexpr int SMEM = OFF_S + MAX_NPB * 4 + 1024;
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(2 * NST <= 32, "two lanes per stage");
+};
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -555,10 +559,14 @@ __device__ __forceinline__ void commit_both(uint64_t* bar) {
 }
 }  // namespace pair
 
-template <bool DEBUG_P, int YMODE>
+template <int PBN, bool DEBUG_P, int YMODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     gemm_f8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g) {
     using namespace pair;
+    using C = PCfg<PBN>;
+    constexpr int BN = C::BN, BNH = C::BNH, KPS = C::KPS, A_TILE = C::A_TILE, B_TILE = C::B_TILE;
+    constexpr int A_STAGE = C::A_STAGE, B_STAGE = C::B_STAGE, STAGE = C::STAGE, NST = C::NST, NBUF = C::NBUF;
+    constexpr int OFF_B = C::OFF_B, OFF_BAR = C::OFF_BAR, OFF_S = C::OFF_S;
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -838,17 +846,20 @@ static bool make_map_kblocks(CUtensorMap* map, const void* base, uint64_t K, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int PBN>
 static cudaError_t launch_pair(const GemmF8Launch& gl, const Args& a, int nsm) {
     using namespace pair;
+    using C = PCfg<PBN>;
+    constexpr int BN = C::BN, BNH = C::BNH, KPS = C::KPS, SMEM = C::SMEM;
     CUtensorMap tmA, tmB;
     if (!make_map_kblocks(&tmA, gl.A, (uint64_t)gl.K, (uint64_t)gl.M, BM, KPS)) return cudaErrorInvalidValue;
     if (!make_map_kblocks(&tmB, gl.B, (uint64_t)gl.K, (uint64_t)gl.N, BNH, KPS)) return cudaErrorInvalidValue;
     const int ntiles = ((gl.M + 2 * BM - 1) / (2 * BM)) * ((gl.N + BN - 1) / BN);
     const int v = gl.P ? 0 : 1 + gl.ymode;
-    auto kern = v == 0 ? gemm_f8_pair_kernel<true, kYF32>
-                : v == 1 ? gemm_f8_pair_kernel<false, kYF32>
-                : v == 2 ? gemm_f8_pair_kernel<false, kYBF16>
-                         : gemm_f8_pair_kernel<false, kYSiluMul>;
+    auto kern = v == 0 ? gemm_f8_pair_kernel<PBN, true, kYF32>
+                : v == 1 ? gemm_f8_pair_kernel<PBN, false, kYF32>
+                : v == 2 ? gemm_f8_pair_kernel<PBN, false, kYBF16>
+                         : gemm_f8_pair_kernel<PBN, false, kYSiluMul>;
     static KernelSetup setup[4];
     static int maxc_cache[4][16] = {};
     int occ = 0;
@@ -878,11 +889,14 @@ static cudaError_t launch_pair(const GemmF8Launch& gl, const Args& a, int nsm) {
 }  // namespace f8
 
 int gemm_f8_pick_bn(int M, int N, int nsm) {
-    // 256 x 256 pair tiles (returned as 512) read the fewest operand bytes per
-    // output; take them when there are enough of them to occupy the SMs.
-    // Otherwise 256-column tiles, unless 128-column ones fill more SMs.
+    // 256 x 256 pair tiles (returned as kPickPair256) read the fewest operand bytes
+    // per output; take them when there are enough of them to occupy the SMs.  Then
+    // 256 x 128 pair tiles (kPickPair128) when they fill three quarters of the SMs.
+    // Otherwise one-CTA 256-column tiles, unless 128-column ones fill more SMs.
     const long tp = (long)((M + 255) / 256) * ((N + 255) / 256);
-    if (2 * tp >= nsm) return 512;
+    if (2 * tp >= nsm) return kPickPair256;
+    const long tp128 = (long)((M + 255) / 256) * ((N + 127) / 128);
+    if (8 * tp128 >= 3 * (long)nsm) return kPickPair128;
     const int nmb = (M + f8::BM - 1) / f8::BM;
     const long t256 = (long)nmb * ((N + 255) / 256);
     const long t128 = (long)nmb * ((N + 127) / 128);
@@ -907,7 +921,8 @@ cudaError_t launch_gemm_f8(const GemmF8Launch& gl) {
     a.limit_ns = kWaitLimitNs;
     const int nsm = device_sm_count();
     const int bn = gl.bn ? gl.bn : gemm_f8_pick_bn(gl.M, gl.N, nsm);
-    if (bn == 512) return f8::launch_pair(gl, a, nsm);
+    if (bn == kPickPair256) return f8::launch_pair<256>(gl, a, nsm);
+    if (bn == kPickPair128) return f8::launch_pair<128>(gl, a, nsm);
     return bn == 128 ? launch_bn<128>(gl, a, nsm) : launch_bn<256>(gl, a, nsm);
 }
 

@@ -141,6 +141,10 @@ struct GemmF8Launch {
     cudaStream_t stream;
 };
 cudaError_t launch_gemm_f8(const GemmF8Launch& gl);
+// Tile choice of the fp8 GEMM: 128 or 256 (one CTA, 128 rows x that many
+// columns), or a CTA pair of 256 rows x 256 / 128 columns.
+constexpr int kPickPair256 = 512;
+constexpr int kPickPair128 = 640;
 int gemm_f8_pick_bn(int M, int N, int nsm);
 // Packed INT4 rows [rows, K/2] -> e4m3 codes [rows, K], natural k order.
 cudaError_t launch_expand_e4m3(const uint8_t* q, uint8_t* out, int rows, int K, cudaStream_t stream);

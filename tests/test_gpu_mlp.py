@@ -123,12 +123,12 @@ def test_mlp_block_quality_bounded(rrs):
     assert all(np.isfinite(v) and v < 0.5 for v in errs.values()), errs
 
 
-@pytest.mark.parametrize("M,F,K", [(512, 9472, 512), (130, 260, 256), (64, 1000, 384)])
+@pytest.mark.parametrize("M,F,K", [(512, 9472, 512), (130, 260, 256), (64, 1000, 384), (2048, 512, 256)])
 def test_gate_up_gemm_with_fused_silu_mul(rrs, M, F, K):
     """RRS_Y_SILU_MUL: the fp8 gate/up GEMM over interleaved weight rows writes H directly;
     it must equal, bit for bit, rrs_silu_mul applied to the same GEMM's fp32 output with
-    its columns de-interleaved into [gate | up] (the shapes take the CTA-pair kernel and
-    the single-CTA one, with ragged edges)."""
+    its columns de-interleaved into [gate | up] (the shapes take the 256 x 256 and
+    256 x 128 CTA-pair kernels and the single-CTA one, with ragged edges)."""
     G = 128
     rng = np.random.default_rng(M + F)
     qX = torch.from_numpy(rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)).to(DEV)

@@ -149,7 +149,10 @@ def test_partials_bit_exact_expanded_weights(rrs, M, N, K, G):
 
 # Shapes with at least 74 tiles of 256 x 256 take the CTA-pair kernel of the fp8
 # GEMM; ragged M and N (not multiples of 256) exercise its edge tiles.
-PAIR_SHAPES = [(300, 19016, 384, 128), (512, 18944, 512, 256), (260, 20480, 256, 256)]
+# 256 x 256 CTA-pair tiles (the first three) and 256 x 128 pair tiles (the last three,
+# narrow N: k/v-like), with ragged edges
+PAIR_SHAPES = [(300, 19016, 384, 128), (512, 18944, 512, 256), (260, 20480, 256, 256),
+               (2048, 1024, 512, 128), (1900, 1000, 384, 128), (2100, 1200, 256, 256)]
 
 
 @pytest.mark.parametrize("M,N,K,G", PAIR_SHAPES)
