@@ -74,7 +74,8 @@ constexpr int kPrefetchUnits = 24;            // units per CTA asked of L2 up fr
 
 // shared memory: rotation buffers | group of each channel | staged codes |
 // per-team group maxima | divisors, token scales, reduction scratch
-constexpr size_t kOffGrp = (size_t)kMaxChunk * 4;
+constexpr int kPadChunk = kMaxChunk + kMaxChunk / 32;   // rotation buffers, one pad word per 32
+constexpr size_t kOffGrp = (size_t)kPadChunk * 4;
 constexpr size_t kOffAct = kOffGrp + kMaxK;
 constexpr size_t kOffGmx = kOffAct + (size_t)kMaxSlots * kMaxTokens * kActStride;
 constexpr size_t kOffPerm = kOffGmx + (size_t)kWarps * kMaxGroups * 4;
@@ -160,26 +161,30 @@ __device__ __forceinline__ int rot_index(int b0, int nb, int tt, int r) {
     return ((other >> b0) << (b0 + nb)) | (lo << b0) | (other & ((1 << b0) - 1));
 }
 
+// Buffer position of element i: one pad word after every 32, so that the
+// power-of-two strides of the rounds fall on different banks.
+__device__ __forceinline__ int padi(int i) { return i + (i >> 5); }
+
 // The thread's sixteen elements to / from the buffer in a round's layout; a
 // full round (nb = 4) holds elements base + r * 2^b0.
 __device__ __forceinline__ void store_round(float* tb, const float (&v)[kEl], int b0, int nb, int tt) {
     if (nb == 4) {
         const int base = ((tt >> b0) << (b0 + 4)) | (tt & ((1 << b0) - 1));
 #pragma unroll
-        for (int r = 0; r < kEl; ++r) tb[base + (r << b0)] = v[r];
+        for (int r = 0; r < kEl; ++r) tb[padi(base + (r << b0))] = v[r];
     } else {
 #pragma unroll
-        for (int r = 0; r < kEl; ++r) tb[rot_index(b0, nb, tt, r)] = v[r];
+        for (int r = 0; r < kEl; ++r) tb[padi(rot_index(b0, nb, tt, r))] = v[r];
     }
 }
 __device__ __forceinline__ void load_round(const float* tb, float (&v)[kEl], int b0, int nb, int tt) {
     if (nb == 4) {
         const int base = ((tt >> b0) << (b0 + 4)) | (tt & ((1 << b0) - 1));
 #pragma unroll
-        for (int r = 0; r < kEl; ++r) v[r] = tb[base + (r << b0)];
+        for (int r = 0; r < kEl; ++r) v[r] = tb[padi(base + (r << b0))];
     } else {
 #pragma unroll
-        for (int r = 0; r < kEl; ++r) v[r] = tb[rot_index(b0, nb, tt, r)];
+        for (int r = 0; r < kEl; ++r) v[r] = tb[padi(rot_index(b0, nb, tt, r))];
     }
 }
 
@@ -203,7 +208,7 @@ __device__ __forceinline__ void rot_stages(float (&v)[kEl], int nb) {
 
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    float* xbuf = reinterpret_cast<float*>(smem);                       // [kMaxChunk]
+    float* xbuf = reinterpret_cast<float*>(smem);                       // [kPadChunk]
     uint8_t* grp = smem + kOffGrp;                                      // [K] group of each channel
     uint8_t* act = smem + kOffAct;                                      // [slots][16][kActStride]
     uint32_t* gmx = reinterpret_cast<uint32_t*>(smem + kOffGmx);        // [warps][kMaxGroups]
@@ -228,6 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
 
     // ---- phase 0: start the weight stream (L2 prefetch) and invert the reorder: channel perm[j] of the rotated row lies in group j / G
     {
+        // the activation rows of this CTA's first rotation items, then weights
+        {
+            const int L0 = L, T0 = L0 / kEl, R0 = kThreads / T0;
+            const int it0 = blockIdx.x * R0 + tid;
+            if (tid < R0 && it0 < M * per_row)
+                prefetch_l2(p.X + (size_t)(it0 / per_row) * K + (size_t)(it0 % per_row) * L0, (uint32_t)L0 * 2);
+        }
         const int npf = min(u1 - u0, kPrefetchUnits);
         for (int e = tid; e < npf * 16; e += kThreads) {
             const int u = u0 + e / 16;
@@ -264,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
         const int T = L / kEl;
         const int R = kThreads / T;
         const int team = tid / T, tt = tid % T;
-        float* tb = xbuf + (size_t)team * L;
+        float* tb = xbuf + (size_t)team * (L + L / 32);
         const int wpt = T / 32;                                  // warps per team
         uint32_t* wg = gmx + (size_t)(tid >> 5) * kMaxGroups;    // this warp's group maxima
         const int lgL = 31 - __clz(L);
@@ -324,7 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
                 float* xr = p.Xr + (size_t)t * K + (size_t)chunk * L;
                 const uint8_t* gc = grp + (size_t)chunk * L;
                 for (int c = tt * 4; c < L; c += T * 4) {
-                    const float4 x4 = *reinterpret_cast<const float4*>(tb + c);
+                    const int pc = padi(c);   // c .. c + 3 lie in one 32-word run
+                    const float4 x4 = make_float4(tb[pc], tb[pc + 1], tb[pc + 2], tb[pc + 3]);
                     *reinterpret_cast<float4*>(xr + c) = x4;
                     atomicMax(wg + gc[c], __float_as_uint(fabsf(x4.x)));
                     atomicMax(wg + gc[c + 1], __float_as_uint(fabsf(x4.y)));
@@ -588,7 +601,7 @@ bool decode_supported(int M, int N, int K, int G, int n) {
 
 // Where the single launch is the faster form (measured on the 70B decode layers):
 // few tokens, or a weight stream large enough to hide the activation phases.
-bool decode_preferred(int M, int N, int K) { return M <= 4 || (long long)N * K >= (1LL << 27); }
+bool decode_preferred(int M, int N, int K) { return M <= 8 || (long long)N * K >= (1LL << 27); }
 
 // Workspace bytes after the 256-byte header: X_rot, the per-item group maxima
 // and the per-chunk sums, each 256-byte aligned.

@@ -41,8 +41,9 @@ def min_workspace(M, K):
     return torch.zeros(256 + (M * K + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
 
 
-def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
-    """Runs the CUDA path and the oracle on the same inputs and compares."""
+def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True, pool=False):
+    """Runs the CUDA path and the oracle on the same inputs and compares (Y on the
+    listed rows, or every row; pool=True computes the oracle's rows in worker processes)."""
     K = X.shape[1]
     unit = bool(flags & rrs.FORCE_UNIT_SCALES)
     n_eff = 1 if flags & rrs.NO_ROTATE else n
@@ -69,7 +70,11 @@ def run_layer(rrs, X, W, perm, G, n, flags=0, rows=None, check_y=True):
     assert_bits_equal(sw, osw, "scale_w")
     assert_bits_equal(qW, oqW, "qW")
     if check_y:
-        Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
+        if pool and rows is None:
+            from _oracle_pool import linear_rows_all
+            Yo, B = linear_rows_all(oqX, os_, ost, oqW, osw, G)
+        else:
+            Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, G, rows=rows)
         for Yt, what in ((Y, "Y"), (Y8, "Y (expanded weights)")):
             Yg = Yt.cpu().numpy() if rows is None else Yt.cpu().numpy()[rows]
             ok = oracle.y_tolerance_ok(Yg, Yo, B)
@@ -371,9 +376,15 @@ def _sample_rows(M, st, k=48, seed=0):
 
 @pytest.mark.parametrize("name", ["llama3_8b_kv", "llama3_8b_qo", "llama3_8b_gateup", "llama3_8b_down"])
 def test_llama3_8b_layers(rrs, name):
+    """Every code and scale; Y on every row for q/o and k/v (the oracle's rows in
+    worker processes), on sampled rows (the largest-scale tokens among them) for the
+    wider gate/up and down layers."""
     L = wl.LAYERS[name]
     X, W = wl.make_activations(L), wl.make_weights(L)
     perm = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(L, sample=1, M=512), L.had_block))
+    if L.N <= 4096 and L.K <= 4096:
+        run_layer(rrs, X, W, perm, L.G, L.had_block, rows=None, pool=True)
+        return
     _, _, _, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
     rows = _sample_rows(L.M, ost, k=24 if L.N > 8192 else 48)
     run_layer(rrs, X, W, perm, L.G, L.had_block, rows=rows)
