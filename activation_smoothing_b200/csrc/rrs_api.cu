@@ -593,6 +593,12 @@ rrs_status rrs_kv_quant(const void* KV, int T, int H, int D, uint8_t* q, float* 
     if (D < 128 || D > kMaxHadamard)
         return fail(RRS_ERR_UNSUPPORTED, "D = %d: the CUDA path takes head sizes 128..%d", D, kMaxHadamard);
     if (flags != 0) return fail(RRS_ERR_INVALID_ARG, "rrs_kv_quant takes no flags (got 0x%x)", flags);
+    if (rrs::kv_quant_warp_supported(D)) {
+        cudaError_t e = rrs::launch_kv_quant_warp(KV, (size_t)T * H, D, (float)(1.0 / std::sqrt((double)D)), q, scale,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "KV quantise kernel");
+        return RRS_OK;
+    }
     rrs::PrepLaunch pl{};
     pl.X = KV;
     pl.rows = T * H;

@@ -85,6 +85,10 @@ bool prep_fast_supported(int K, int n);
 int prep_fast_rows_per_cta(int K);
 cudaError_t launch_prep_fast(const PrepFastLaunch& pl, cudaStream_t stream);
 // KV cache: out fp16 [rows, D] = code * scale[row] from packed INT4 q [rows, D/2].
+// KV-cache quantisation for head sizes 128, 256, 512: 32 channels per lane.
+bool kv_quant_warp_supported(int D);
+cudaError_t launch_kv_quant_warp(const void* kv, size_t rows, int D, float c_n, uint8_t* q, float* scale,
+                                 cudaStream_t stream);
 cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows, int D, void* out,
                               cudaStream_t stream);
 // p[0..n) = v.

@@ -42,7 +42,121 @@ __global__ void dequant_kernel(const uint8_t* q, const float* scale, size_t rows
     }
 }
 
+// Quantisation of head vectors of D channels by LPV = D / 32 lanes each (32
+// channels per lane, in registers; a warp takes 32 / LPV vectors at a time).  The
+// normalised Hadamard transform runs in the library's stage order (h = 1, 2, 4,
+// ...; pair (a + b, a - b), a the lower index): the stages h < 32 inside a lane,
+// the stages h = 32, 64, ... across the vector's lanes by shuffles (the lane with
+// the clear bit holds the lower index).  Then x = fl(c_n v), amax = max |x| over
+// the vector, scale = amax / 7, q = clamp(rint(x / scale), -8, 7), the division
+// correctly rounded by Markstein's correction as in the activation kernels (a
+// zero scale gives zero codes).
+template <int LPV>
+__global__ void __launch_bounds__(256) quant_kernel(const __half* kv, size_t rows, float c_n, uint8_t* q,
+                                                    float* scale) {
+    constexpr int E = 32;                         // channels per lane, held as 16 float2
+    constexpr int D = LPV * E;
+    constexpr int VPW = 32 / LPV;                 // vectors per warp per pass
+    constexpr float kMagic = 12582912.0f;         // 1.5 * 2^23: adding it rounds to an integer, half to even
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPV;                   // this lane's part of its vector
+    const size_t warp0 = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5;
+    const size_t nwarps = (gridDim.x * (size_t)blockDim.x) >> 5;
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    for (size_t rb = warp0 * VPW; rb < rows; rb += nwarps * VPW) {
+        const size_t r = rb + lane / LPV;
+        const bool live = r < rows;
+        float2 v[E / 2];
+        const __half* src = kv + (live ? r : 0) * D + (size_t)sub * E;
+#pragma unroll
+        for (int c = 0; c < E; c += 8) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src + c);
+            const __half2* h = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[c / 2 + k] = __half22float2(h[k]);
+        }
+        // stage h = 1: the two channels of one float2
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) {
+            const float a = v[i].x, b = v[i].y;
+            v[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+        }
+        // stages h = 2 .. 16: pairs of float2, lane by lane with packed add / sub
+        // (a - b as fma(b, -1, a), which is exactly RN(a - b))
+#pragma unroll
+        for (int hh = 1; hh < E / 2; hh <<= 1) {
+#pragma unroll
+            for (int i = 0; i < E / 2; ++i) {
+                if (!(i & hh)) {
+                    const float2 a = v[i], b = v[i + hh];
+                    v[i] = __fadd2_rn(a, b);
+                    v[i + hh] = __ffma2_rn(b, neg1, a);
+                }
+            }
+        }
+        // stages h = 32, 64, ...: the partner lane's value p; the lower lane keeps
+        // RN(v + p), the upper RN(p - v): both are fma(v, +-1, p)
+#pragma unroll
+        for (int m = 1; m < LPV; m <<= 1) {
+            const float sg = (lane & m) ? -1.0f : 1.0f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int i = 0; i < E / 2; ++i) {
+                const float2 pv = make_float2(__shfl_xor_sync(0xFFFFFFFFu, v[i].x, m),
+                                              __shfl_xor_sync(0xFFFFFFFFu, v[i].y, m));
+                v[i] = __ffma2_rn(v[i], sg2, pv);
+            }
+        }
+        const float2 c2 = make_float2(c_n, c_n);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) {
+            v[i] = __fmul2_rn(v[i], c2);
+            amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        }
+#pragma unroll
+        for (int m = 1; m < LPV; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, m));
+        const float sc = __fdiv_rn(amax, 7.0f);
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
+        if (sc != 0.0f) {
+            // |x| / scale <= 7 (to within an ulp: scale = RN(amax / 7)), so rint needs no clamp
+            const float ys = __frcp_rn(sc);
+            const float2 ns2 = make_float2(-sc, -sc), ys2 = make_float2(ys, ys);
+            const float2 magic2 = make_float2(kMagic, kMagic);
+#pragma unroll
+            for (int i = 0; i < E / 2; ++i) {
+                const float2 z = __fadd2_rn(div_markstein(v[i], ns2, ys2), magic2);   // low byte: the code
+                const uint32_t b = (__float_as_uint(z.x) & 15u) | ((__float_as_uint(z.y) & 15u) << 4);
+                packed[i / 4] |= b << (8 * (i % 4));
+            }
+        }
+        if (live) {
+            *reinterpret_cast<uint4*>(q + r * (D / 2) + (size_t)sub * (E / 2)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            if (sub == 0) scale[r] = sc;
+        }
+    }
+}
+
 }  // namespace kv
+
+bool kv_quant_warp_supported(int D) { return D == 128 || D == 256 || D == 512; }
+
+cudaError_t launch_kv_quant_warp(const void* kv, size_t rows, int D, float c_n, uint8_t* q, float* scale,
+                                 cudaStream_t st) {
+    const int LPV = D / 32;
+    const size_t per_block = 8 * (size_t)(32 / LPV);        // vectors per block per pass
+    size_t blocks = (rows + per_block - 1) / per_block;
+    const size_t cap = (size_t)device_sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const __half* x = reinterpret_cast<const __half*>(kv);
+    if (LPV == 4) kv::quant_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(x, rows, c_n, q, scale);
+    else if (LPV == 8) kv::quant_kernel<8><<<(unsigned)blocks, 256, 0, st>>>(x, rows, c_n, q, scale);
+    else if (LPV == 16) kv::quant_kernel<16><<<(unsigned)blocks, 256, 0, st>>>(x, rows, c_n, q, scale);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
 
 cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows, int D, void* out,
                               cudaStream_t st) {

@@ -28,7 +28,10 @@ def _kv(T, H, D, seed):
     return x.clamp(-65504, 65504).to(torch.float16)
 
 
-@pytest.mark.parametrize("T,H,D", [(64, 8, 128), (33, 4, 256), (1, 1, 128), (517, 8, 128), (7, 2, 512)])
+# D = 128, 256, 512 take the warp-per-vector kernel (with vector counts that are not a
+# multiple of its per-warp batch), D = 1024 the general activation kernels
+@pytest.mark.parametrize("T,H,D", [(64, 8, 128), (33, 4, 256), (1, 1, 128), (517, 8, 128), (7, 2, 512),
+                                   (3, 3, 128), (5, 2, 1024)])
 def test_kv_quant_bit_exact(rrs, T, H, D):
     x = _kv(T, H, D, T * 7 + D)
     q, sc = rrs.kv_quant(x.to(DEV))
