@@ -42,6 +42,31 @@ __global__ void dequant_kernel(const uint8_t* q, const float* scale, size_t rows
     }
 }
 
+// The same for D a power of two >= 32: 32 outputs per thread (one 16-byte load of
+// codes, four 16-byte stores), the row from a shift.
+__device__ __forceinline__ uint32_t half2_codes(uint32_t byte, float sc) {
+    const int lo = (int)(byte & 0x0Fu) - (int)((byte & 0x08u) << 1);
+    const int hi = (int)((byte >> 4) & 0x0Fu) - (int)((byte & 0x80u) >> 3);
+    const __half2 h = __floats2half2_rn(__fmul_rn((float)lo, sc), __fmul_rn((float)hi, sc));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__global__ void dequant32_kernel(const uint8_t* q, const float* scale, size_t rows, int lg_chunks, __half* out) {
+    const size_t total = rows << lg_chunks;      // 32-output chunks
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const uint4 w = reinterpret_cast<const uint4*>(q)[i];
+        const float sc = scale[i >> lg_chunks];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint4* dst = reinterpret_cast<uint4*>(out) + 4 * i;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t x = ws[k];
+            dst[k] = make_uint4(half2_codes(x & 0xFFu, sc), half2_codes((x >> 8) & 0xFFu, sc),
+                                half2_codes((x >> 16) & 0xFFu, sc), half2_codes(x >> 24, sc));
+        }
+    }
+}
+
 // Quantisation of head vectors of D channels by LPV = D / 32 lanes each (32
 // channels per lane, in registers; a warp takes 32 / LPV vectors at a time).  The
 // normalised Hadamard transform runs in the library's stage order (h = 1, 2, 4,
@@ -160,9 +185,19 @@ cudaError_t launch_kv_quant_warp(const void* kv, size_t rows, int D, float c_n, 
 
 cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows, int D, void* out,
                               cudaStream_t st) {
+    const size_t cap = (size_t)device_sm_count() * 16;
+    if (D >= 32 && (D & (D - 1)) == 0) {
+        int lg = 0;
+        while ((32 << lg) < D) ++lg;
+        const size_t total = rows << lg;
+        size_t blocks = (total + 255) / 256;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+        kv::dequant32_kernel<<<(unsigned)blocks, 256, 0, st>>>(q, scale, rows, lg, reinterpret_cast<__half*>(out));
+        return cudaGetLastError();
+    }
     const size_t total = rows * (size_t)(D / 8);
     size_t blocks = (total + 255) / 256;
-    const size_t cap = (size_t)device_sm_count() * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     kv::dequant_kernel<<<(unsigned)blocks, 256, 0, st>>>(q, scale, rows, D, reinterpret_cast<__half*>(out));

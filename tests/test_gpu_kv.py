@@ -49,3 +49,18 @@ def test_kv_quant_rejects_bad_sizes(rrs):
     with pytest.raises(rrs.RRSError) as e:
         rrs.kv_quant(x)
     assert e.value.status_name == "RRS_ERR_UNSUPPORTED"
+
+
+@pytest.mark.parametrize("T,H,D", [(9, 3, 40), (4, 2, 32), (130, 1, 64)])
+def test_kv_dequant_of_any_codes(rrs, T, H, D):
+    """The way back for head sizes the quantiser does not take (D a multiple of 8,
+    or a power of two below 128): fp16(code * scale) against the oracle's fp32
+    reconstruction rounded to fp16."""
+    rng = np.random.default_rng(T * H + D)
+    q = rng.integers(0, 256, size=(T, H, D // 2), dtype=np.uint8)
+    sc = (rng.random((T, H), dtype=np.float32) * 3).astype(np.float32)
+    sc[0, 0] = 0.0
+    back = rrs.kv_dequant(torch.from_numpy(q).to(DEV), torch.from_numpy(sc).to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.kv_dequant(q, sc).astype(np.float16)
+    assert np.array_equal(back.cpu().numpy().view(np.uint16), ref.view(np.uint16))
