@@ -206,6 +206,9 @@ __device__ __forceinline__ void rot_stages(float (&v)[kEl], int nb) {
     }
 }
 
+// TWO: more than 8 tokens (a second 8-column MMA tile); a separate form keeps
+// the one-token kernel smaller (its code runs once per launch, fetched cold).
+template <bool TWO>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
     extern __shared__ __align__(16) unsigned char smem[];
     float* xbuf = reinterpret_cast<float*>(smem);                       // [kPadChunk]
@@ -410,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
         // word, the codes of the even channels and of the odd ones as int8x4 words of
         // 16 * code.  A thread takes one word and four tokens (all loads at once).
         const int nslot = u1 > u0 ? (u1 - 1) / p.RT - kc_first + 1 : 0;
-        const int TOK = M <= 8 ? 8 : 16;
+        constexpr int TOK = TWO ? 16 : 8;
+        constexpr int NQ = TOK / 4;                // token subsets per staged word
         for (int e = tid; e < nslot * kActWords * 4; e += kThreads) {
             const int wi = e % kActWords;
             const int tq = (e / kActWords) % 4;
@@ -420,17 +424,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
             const int4 pb = *reinterpret_cast<const int4*>(pslot + sl * KC + 8 * wi + 4);
             const int src[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
             const float sd = s_sm[j0 / G], yd = ys_sm[j0 / G];
-            float x[4][8];
+            float x[NQ][8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < NQ; ++q) {
                 const int t = tq + 4 * q;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) x[q][c] = t < M ? __ldcg(p.Xr + (size_t)t * K + src[c]) : 0.0f;
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < NQ; ++q) {
                 const int t = tq + 4 * q;
-                if (t >= TOK) continue;
                 uint32_t ev = 0, od = 0;
                 if (t < M) {
 #pragma unroll
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const Args p) {
         const int warp = tid >> 5, lane = tid & 31;
         const int gq = lane >> 2, tq = lane & 3;
         const int gpb = G / 128;                   // MMA blocks per group (G divides KC)
-        const bool two = M > 8;
+        constexpr bool two = TWO;
         // A unit's weights in two register halves (blocks 0-3, 4-7): rows gq (a) and
         // gq + 8 (b) of the tile.  The next unit's halves are loaded as soon as this
         // unit's are used.
@@ -601,7 +604,7 @@ bool decode_supported(int M, int N, int K, int G, int n) {
 
 // Where the single launch is the faster form (measured on the 70B decode layers):
 // few tokens, or a weight stream large enough to hide the activation phases.
-bool decode_preferred(int M, int N, int K) { return M <= 8 || (long long)N * K >= (1LL << 27); }
+bool decode_preferred(int M, int N, int K) { return M <= 6 || (long long)N * K >= (1LL << 27); }
 
 // Workspace bytes after the 256-byte header: X_rot, the per-item group maxima
 // and the per-chunk sums, each 256-byte aligned.
@@ -613,9 +616,11 @@ size_t decode_ws_bytes(int M, int N, int K) {
 
 cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t st) {
     using namespace dec;
-    static KernelSetup setup;
+    static KernelSetup setup[2];
+    const bool two = dl.M > 8;
+    const auto kern = two ? decode_kernel<true> : decode_kernel<false>;
     int occ = 0;
-    cudaError_t e = kernel_setup(reinterpret_cast<const void*>(decode_kernel), kThreads, kSmemBytes, setup, &occ);
+    cudaError_t e = kernel_setup(reinterpret_cast<const void*>(kern), kThreads, kSmemBytes, setup[two ? 1 : 0], &occ);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
     const int grid = decode_grid();
@@ -650,7 +655,7 @@ cudaError_t launch_decode(const DecodeLaunch& dl, cudaStream_t st) {
     a.err = dl.err;
     a.limit_ns = kWaitLimitNs;
     void* params[] = {&a};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_kernel), dim3(grid), dim3(kThreads), params,
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(kThreads), params,
                                        kSmemBytes, st);
 }
 

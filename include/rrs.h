@@ -113,7 +113,7 @@ typedef enum {
 #define RRS_ONE_LAUNCH 64u       /* rrs_linear, rrs_linear_from_host: for M <= 16 with packed
                                     weights, always take the single-launch layer where the
                                     shape allows it.  Without it the single launch is taken
-                                    only where it is the faster of the two forms: M <= 8, or
+                                    only where it is the faster of the two forms: M <= 6, or
                                     N * K >= 2^27 (the weight stream then outweighs the
                                     fixed cost of the in-kernel activation phases). */
 
