@@ -1,21 +1,26 @@
 // rrs_prep_fast.cu -- online activation path for K a multiple of 2048 (every
-// LLaMA projection shape): one cooperative persistent kernel in two phases.
+// LLaMA projection shape): one cooperative persistent kernel in two phases
+// (the kernel itself is in rrs_act.cuh, instantiated in rrs_act_*.cu).
 //
-//   phase A   X (fp16) -> Hadamard rotation and reorder gather of every row
-//             this CTA owns; each thread keeps the largest |X'| of its outputs
-//             (all in one group), and the CTA's group maxima go into one row of
-//             a per-CTA table in the workspace
+//   phase A   X (fp16) -> Hadamard rotation of every row this CTA owns; each
+//             thread keeps, per register, the largest |v| of its channel over
+//             its rows, and at the end the CTA's per-channel maxima are gathered
+//             by the reorder into its row of a group-maxima table in the
+//             workspace (fl(c_n |v|) is monotone in |v|, so c_n is applied once)
 //   barrier   a grid-wide barrier (bounded wait); every CTA then reduces the
 //             table: s[g] = max over all tokens and group channels of |X'|
 //   phase B   X again (an L2 hit) -> the same rotation bit for bit, reorder
 //             gather, division by s_g, per-token INT4 quantisation; writes qX
-//             (packed), scale_t and, if asked, the GEMM operand.  When every
-//             team owns at most one row (decode token counts), the rotated row
-//             stays in shared memory across the barrier and is not recomputed.
+//             (packed), scale_t and the GEMM operand (e4m3 or int8).  When every
+//             team owns at most one row (decode token counts), phase A keeps the
+//             rotated row in shared memory and phase B does not recompute it.
 //
 // Nothing of size M x K passes between the phases: the rotation is recomputed
-// (or kept on chip) instead of stored.
-
+// (or kept on chip) instead of stored.  The host picks one of eight kernel forms
+// (256 or 512 threads, rows kept or not, e4m3 or int8 operand), each a smaller
+// kernel: in a layer sequence the kernel follows a GEMM and its code is fetched
+// cold, so code size is time.
+//
 // Work split: a team of T = K/64 threads (a multiple of 32) owns one row at a
 // time; each thread holds 64 elements.  Rotation rounds: up to 6 butterfly
 // stages on the 64 registers (f32x2 packed add/sub for every stage but the
@@ -53,7 +58,8 @@ extern template cudaError_t launch_act<11>(const ActArgs&, bool, int, size_t, in
 extern template cudaError_t launch_act<12>(const ActArgs&, bool, int, size_t, int, cudaStream_t);
 extern template cudaError_t launch_act<13>(const ActArgs&, bool, int, size_t, int, cudaStream_t);
 
-// Packed INT4 rows -> int8 GEMM operand rows (same k order as smooth_quant_kernel).
+// Packed INT4 rows -> int8 GEMM operand rows (the k order of the activation
+// kernel's int8 operand: 0, 2, 4, 6, 1, 3, 5, 7 within each 8 channels).
 __global__ void expand_kernel(const uint8_t* qX, int8_t* qX8, size_t nwords) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nwords; i += (size_t)gridDim.x * blockDim.x) {
         const uint32_t w = reinterpret_cast<const uint32_t*>(qX)[i];

@@ -197,3 +197,32 @@ def test_full_70b_decode_sizes(rrs, name):
     d = (Y - Y2).abs()
     assert (d <= 1e-3 * Y2.abs() + 1e-6 * Y2.abs().max()).all()
     assert (torch.linalg.norm(Y - Y2) / torch.linalg.norm(Y2)).item() < 1e-5
+
+
+@pytest.mark.parametrize("M,one_launch", [(1, True), (6, True), (12, False)])
+def test_default_choice_of_form(rrs, M, one_launch):
+    """Without RRS_ONE_LAUNCH, rrs_linear takes the single launch for M <= 6 (or a
+    large weight stream) and the two launches otherwise; the rotated rows left in
+    the workspace show which ran.  Both give the oracle's codes and Y."""
+    L = wl.LAYERS["llama3_8b_qo"]
+    X, W = wl.make_activations(L, sample=M, M=M), wl.make_weights(L, N=256)
+    perm = wl.random_perm(L.K, M)
+    Xd, pd = X.to(DEV), perm.to(DEV)
+    qW, sw = rrs.prepare_weights(W.to(DEV), pd, L.had_block)
+    ws = rrs.make_workspace(M, 256, L.K, L.G, L.had_block)
+    qX = torch.empty((M, L.K // 2), dtype=torch.uint8, device=DEV)
+    s = torch.empty(L.K // L.G, dtype=torch.float32, device=DEV)
+    st = torch.empty(M, dtype=torch.float32, device=DEV)
+    Y = rrs.linear(Xd, qW, sw, pd, L.G, L.had_block, qX=qX, s=s, scale_t=st, ws=ws)
+    rrs.check_workspace(ws)
+    torch.cuda.synchronize()
+    rot = ws[256:256 + M * L.K * 4].view(torch.float32).view(M, L.K).cpu().numpy()
+    same_rot = np.array_equal(rot.view(np.uint32), oracle.rotate(X, L.had_block).view(np.uint32))
+    assert same_rot == one_launch
+    _, oqX, os_, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
+    _same(qX, oqX, "qX")
+    _same(s, os_, "s")
+    _same(st, ost, "scale_t")
+    _, oqW, osw = oracle.prepare_weights(W, L.had_block, perm.numpy())
+    Yo, B = oracle.linear_rows(oqX, os_, ost, oqW, osw, L.G)
+    assert oracle.y_tolerance_ok(Y.cpu().numpy(), Yo, B).all()
