@@ -432,6 +432,9 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     }
     if (!(p.phase & 2)) return;
     __syncthreads();
+    // the GEMM that reads this kernel's outputs may start launching (it waits for
+    // this kernel's completion before reading them)
+    grid_dependents_launch();
 
     // --------------------------------------------------------------- phase B
     it = 0;

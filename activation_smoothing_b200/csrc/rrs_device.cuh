@@ -240,6 +240,13 @@ __device__ __forceinline__ float div_markstein(float a, float nb, float y) {
     return __fmaf_rn(r, y, q0);
 }
 
+// Programmatic dependent launch: the dependent kernel waits here until the
+// kernel before it in the stream has completed and its memory operations are
+// visible (a no-op when it was not launched as a dependent); the primary kernel
+// lets its dependents start launching early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // The gated-MLP activation of one output: silu(g) * u with silu(g) = g / (1 +
 // exp(-g)) in fp32, saturated to +-65504 (the fp16 range the next layer's
 // activation path takes); the caller rounds it to fp16.  One definition for the

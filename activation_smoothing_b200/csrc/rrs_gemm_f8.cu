@@ -356,12 +356,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (!DEBUG_P) {
-        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
-    }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
+    }
+    // launched as a programmatic dependent of the activation kernel: everything
+    // above overlapped its end; its outputs (operand, s, scale_t) are read below
+    grid_dependency_wait();
+    if (!DEBUG_P) {
+        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
     }
     tc_fence_before();
     __syncthreads();
@@ -607,17 +610,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (!DEBUG_P) {
-        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
-    }
     if (warp == MMA_WARP) {
         // both CTAs' warp 2 allocate together: the same columns in both TMEMs
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(512) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    // launched as a programmatic dependent of the activation kernel: everything
+    // above overlapped its end; its outputs (operand, s, scale_t) are read below
+    grid_dependency_wait();
+    if (!DEBUG_P) {
+        for (int i = threadIdx.x; i < NPB; i += blockDim.x) s_sm[i] = g.s[(i * g.PB) / g.G];
+    }
     tc_fence_before();
-    cluster_sync();          // barriers of both CTAs initialised and visible, TMEM allocated
+    cluster_sync();          // barriers of both CTAs initialised and visible, TMEM allocated, s staged
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -781,6 +787,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
 }
 
+// A launch that may begin while the previous kernel in the stream finishes
+// (programmatic dependent launch); the kernel waits with griddepcontrol.wait
+// before it reads what that kernel wrote.  After any other stream operation it
+// behaves as a plain launch.
+template <typename Kern>
+static cudaError_t launch_dependent(Kern kern, dim3 grid, int threads, int smem, cudaStream_t st,
+                                   const CUtensorMap& tmA, const CUtensorMap& tmB, const Args& a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -827,8 +853,7 @@ static cudaError_t launch_bn(const GemmF8Launch& gl, const Args& a, int nsm) {
     int occ = 0;
     cudaError_t e = kernel_setup(reinterpret_cast<const void*>(kern), NTHREADS, C::SMEM, setup[v], &occ);
     if (e != cudaSuccess) return e;
-    kern<<<grid, NTHREADS, C::SMEM, gl.stream>>>(tmA, tmB, a);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), NTHREADS, C::SMEM, gl.stream, tmA, tmB, a);
 }
 
 // 3-D view {128 bytes, rows, K / 128} of a [rows, K] uint8 operand (k-block
@@ -882,8 +907,7 @@ static cudaError_t launch_pair(const GemmF8Launch& gl, const Args& a, int nsm) {
         if (dev >= 0 && dev < 16) maxc_cache[v][dev] = maxc;
     }
     const int pairs = ntiles < maxc ? ntiles : maxc;
-    kern<<<2 * pairs, NTHREADS, SMEM, gl.stream>>>(tmA, tmB, a);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(2 * pairs), NTHREADS, SMEM, gl.stream, tmA, tmB, a);
 }
 
 }  // namespace f8
