@@ -539,3 +539,38 @@ def test_one_hadamard_size_at_two_row_lengths_in_sequence(rrs):
     assert_bits_equal(s, os_, "s")
     assert_bits_equal(st, ost, "scale_t")
     assert_bits_equal(qX, oqX, "qX")
+
+
+@pytest.mark.parametrize("flags", [0, "expanded"])
+def test_group_larger_than_a_promotion_block(rrs, flags):
+    """G = 6144 (K = 12288): the GEMM promotes in blocks of 3072 channels (the largest
+    multiple of 128 that divides G and is at most 4096); every group's P_g must still be
+    the oracle's, on the packed and the fp8 kernel, and Y within the tolerance."""
+    M, N, K, G = 64, 256, 12288, 6144
+    rng = np.random.default_rng(6144)
+    qX = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    qWd = torch.from_numpy(qW).to(DEV)
+    fl = rrs.W_EXPANDED if flags == "expanded" else 0
+    qWg = rrs.expand_weights(qWd) if fl else qWd
+    P = rrs.w4a4_gemm_debug_partials(torch.from_numpy(qX).to(DEV), qWg, G, flags=fl)
+    assert_bits_equal(P, oracle.group_partials(qX, qW, G), "P_g (G = 6144)")
+    s = (rng.random(K // G, dtype=np.float32) + 0.5).astype(np.float32)
+    st = rng.random(M, dtype=np.float32)
+    sw = rng.random(N, dtype=np.float32)
+    Y = rrs.w4a4_gemm(torch.from_numpy(qX).to(DEV), torch.from_numpy(s).to(DEV), torch.from_numpy(st).to(DEV),
+                      qWg, torch.from_numpy(sw).to(DEV), G, flags=fl)
+    torch.cuda.synchronize()
+    Yo, B = oracle.linear_rows(qX, s, st, qW, sw, G)
+    assert oracle.y_tolerance_ok(Y.cpu().numpy(), Yo, B).all()
+
+
+def test_largest_k(rrs):
+    """K = 32768 (four Hadamard blocks of 8192): the one-launch activation kernel's
+    shared memory would not fit, so the general kernels take it; codes and scales
+    bit-exact, and the layer's Y within the tolerance."""
+    M, N, K, G, n = 8, 128, 32768, 128, 8192
+    L = wl.Layer("k32768", M, K, N, G, n, seed=32768)
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    perm = wl.random_perm(K, 5)
+    run_layer(rrs, X, W, perm, G, n, rows=None)
