@@ -31,6 +31,13 @@ def test_header_declares_the_four_core_calls():
         assert n in names
 
 
+def test_binding_constants_match_the_header():
+    from activation_smoothing_b200 import _binding as b
+    defs = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define RRS_(\w+) (\d+)u", open(HEADER).read())}
+    for name in ("NO_ROTATE", "FORCE_UNIT_SCALES", "WS_HOLDS_A8", "W_EXPANDED", "Y_BF16", "Y_SILU_MUL", "ONE_LAUNCH"):
+        assert getattr(b, name) == defs[name], name
+
+
 def test_library_exports_every_declared_symbol(L):
     names = declared_functions()
     assert len(names) >= 10
