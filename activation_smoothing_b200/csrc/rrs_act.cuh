@@ -16,7 +16,12 @@ namespace fast {
 
 constexpr int E = 64;        // elements per thread
 constexpr int LOGE = 6;
-constexpr int CTA = 256;     // threads per CTA when T <= 256
+// Threads per CTA when T <= CTA: as many row teams as fit in 320 threads.  At
+// K = 4096 that is 5 teams (2048 rows on 148 SMs: at most 3 rows per team and
+// phase instead of 4 with 256 threads); 320 threads leave 204 registers each, and
+// 5 row buffers with 3 staging slots fit in shared memory.
+constexpr int CTA = 320;
+constexpr int BIG = 512;     // threads per CTA of the forms for T > CTA (one row team)
 
 __device__ __forceinline__ int swz(int idx) { return idx ^ (((idx >> LOGE) & 7) << 2); }
 
@@ -531,6 +536,7 @@ cudaError_t launch_act(const ActArgs& a, bool e4m3, int threads, size_t smem, in
     const int R = threads / (a.K / E);
     int grid = (a.rows + R - 1) / R;
     const bool big = threads > CTA;
+    if (threads > BIG) return cudaErrorInvalidConfiguration;
     // occupancy is 1 CTA per SM for every form (shared memory); checked below
     if (grid > nsm) grid = nsm;
     if (grid > grid_cap) grid = grid_cap;
@@ -540,8 +546,8 @@ cudaError_t launch_act(const ActArgs& a, bool e4m3, int threads, size_t smem, in
     static const K_t kerns[8] = {
         act_kernel<L, CTA, false, false>, act_kernel<L, CTA, false, true>,
         act_kernel<L, CTA, true, false>, act_kernel<L, CTA, true, true>,
-        act_kernel<L, 2 * CTA, false, false>, act_kernel<L, 2 * CTA, false, true>,
-        act_kernel<L, 2 * CTA, true, false>, act_kernel<L, 2 * CTA, true, true>};
+        act_kernel<L, BIG, false, false>, act_kernel<L, BIG, false, true>,
+        act_kernel<L, BIG, true, false>, act_kernel<L, BIG, true, true>};
     static KernelSetup setup[8];
     const K_t kern = kerns[form];
     int occ = 0;

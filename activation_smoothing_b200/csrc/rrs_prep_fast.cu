@@ -17,7 +17,7 @@
 //
 // Nothing of size M x K passes between the phases: the rotation is recomputed
 // (or kept on chip) instead of stored.  The host picks one of eight kernel forms
-// (256 or 512 threads, rows kept or not, e4m3 or int8 operand), each a smaller
+// (up to 320 or 512 threads, rows kept or not, e4m3 or int8 operand), each a smaller
 // kernel: in a layer sequence the kernel follows a GEMM and its code is fetched
 // cold, so code size is time.
 //
