@@ -342,6 +342,17 @@ def test_edge_shapes(rrs, M, N, K, G, n):
     run_layer(rrs, X, W, wl.random_perm(K, M + N), G, n)
 
 
+@pytest.mark.parametrize("M,K", [(700, 6144), (400, 10240), (9, 10240)])
+def test_activation_kernel_team_layouts(rrs, M, K):
+    """K values whose row teams fill the activation kernel's CTA differently: K = 6144
+    (three teams of 96 threads) and K = 10240 (two teams of 160, 320 threads), with more
+    rows than teams (the rotation recomputed in pass B) and with one row per team (the
+    rotated row kept on chip); Hadamard blocks of 2048."""
+    L = wl.Layer("teams", M, K, 256, 128, 2048, seed=M + K)
+    X, W = wl.make_activations(L), wl.make_weights(L)
+    run_layer(rrs, X, W, wl.random_perm(K, M), 128, 2048, rows=np.unique(np.r_[0:4, M - 4:M, M // 2]))
+
+
 def test_zero_group_and_zero_token(rrs):
     L = wl.Layer("zeros", 40, 512, 256, 128, 512, seed=3)
     X, W = wl.make_activations(L), wl.make_weights(L)
