@@ -42,8 +42,8 @@ __global__ void dequant_kernel(const uint8_t* q, const float* scale, size_t rows
     }
 }
 
-// The same for D a power of two >= 32: 32 outputs per thread (one 16-byte load of
-// codes, four 16-byte stores), the row from a shift.
+// Two codes (one byte: low nibble the even channel) times the vector's scale, as
+// a half2.
 __device__ __forceinline__ uint32_t half2_codes(uint32_t byte, float sc) {
     const int lo = (int)(byte & 0x0Fu) - (int)((byte & 0x08u) << 1);
     const int hi = (int)((byte >> 4) & 0x0Fu) - (int)((byte & 0x80u) >> 3);
@@ -51,18 +51,27 @@ __device__ __forceinline__ uint32_t half2_codes(uint32_t byte, float sc) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void dequant32_kernel(const uint8_t* q, const float* scale, size_t rows, int lg_chunks, __half* out) {
-    const size_t total = rows << lg_chunks;      // 32-output chunks
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const uint4 w = reinterpret_cast<const uint4*>(q)[i];
-        const float sc = scale[i >> lg_chunks];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        uint4* dst = reinterpret_cast<uint4*>(out) + 4 * i;
+// The same for D a power of two >= 32, by 4-byte code words (8 outputs, one
+// 16-byte store): consecutive threads take consecutive words, so a warp reads 128
+// contiguous bytes of codes and writes 512 contiguous bytes of fp16 per
+// instruction (whole sectors); four words per thread and pass are in flight.
+__global__ void dequant_words_kernel(const uint32_t* q, const float* scale, size_t words, int lg_wpr, uint4* out) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t w0 = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w0 < words; w0 += 4 * stride) {
+        uint32_t c[4];
+        float sc[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t x = ws[k];
-            dst[k] = make_uint4(half2_codes(x & 0xFFu, sc), half2_codes((x >> 8) & 0xFFu, sc),
-                                half2_codes((x >> 16) & 0xFFu, sc), half2_codes(x >> 24, sc));
+        for (int j = 0; j < 4; ++j) {
+            const size_t w = w0 + j * stride;
+            c[j] = w < words ? q[w] : 0u;
+            sc[j] = w < words ? scale[w >> lg_wpr] : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const size_t w = w0 + j * stride;
+            if (w < words)
+                out[w] = make_uint4(half2_codes(c[j] & 0xFFu, sc[j]), half2_codes((c[j] >> 8) & 0xFFu, sc[j]),
+                                    half2_codes((c[j] >> 16) & 0xFFu, sc[j]), half2_codes(c[j] >> 24, sc[j]));
         }
     }
 }
@@ -187,13 +196,14 @@ cudaError_t launch_kv_dequant(const uint8_t* q, const float* scale, size_t rows,
                               cudaStream_t st) {
     const size_t cap = (size_t)device_sm_count() * 16;
     if (D >= 32 && (D & (D - 1)) == 0) {
-        int lg = 0;
-        while ((32 << lg) < D) ++lg;
-        const size_t total = rows << lg;
-        size_t blocks = (total + 255) / 256;
+        int lg = 0;                       // log2 of the code words per row (D / 8)
+        while ((8 << lg) < D) ++lg;
+        const size_t words = rows << lg;
+        size_t blocks = (words + 1023) / 1024;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
-        kv::dequant32_kernel<<<(unsigned)blocks, 256, 0, st>>>(q, scale, rows, lg, reinterpret_cast<__half*>(out));
+        kv::dequant_words_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(q), scale, words,
+                                                                    lg, reinterpret_cast<uint4*>(out));
         return cudaGetLastError();
     }
     const size_t total = rows * (size_t)(D / 8);
