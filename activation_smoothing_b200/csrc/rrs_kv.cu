@@ -158,10 +158,18 @@ __global__ void __launch_bounds__(256) quant_kernel(const __half* kv, size_t row
             const float2 ns2 = make_float2(-sc, -sc), ys2 = make_float2(ys, ys);
             const float2 magic2 = make_float2(kMagic, kMagic);
 #pragma unroll
-            for (int i = 0; i < E / 2; ++i) {
-                const float2 z = __fadd2_rn(div_markstein(v[i], ns2, ys2), magic2);   // low byte: the code
-                const uint32_t b = (__float_as_uint(z.x) & 15u) | ((__float_as_uint(z.y) & 15u) << 4);
-                packed[i / 4] |= b << (8 * (i % 4));
+            for (int w = 0; w < 4; ++w) {   // 8 channels (4 float2) per packed word
+                uint32_t ev[4], od[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 z = __fadd2_rn(div_markstein(v[4 * w + h], ns2, ys2), magic2);   // low byte: the code
+                    ev[h] = __float_as_uint(z.x);
+                    od[h] = __float_as_uint(z.y);
+                }
+                // byte h of lo / hi: the code of channel 2h / 2h + 1 of the word
+                const uint32_t lo = __byte_perm(__byte_perm(ev[0], ev[1], 0x0040), __byte_perm(ev[2], ev[3], 0x0040), 0x5410);
+                const uint32_t hi = __byte_perm(__byte_perm(od[0], od[1], 0x0040), __byte_perm(od[2], od[3], 0x0040), 0x5410);
+                packed[w] = (lo & 0x0F0F0F0Fu) | ((hi << 4) & 0xF0F0F0F0u);
             }
         }
         if (live) {
