@@ -105,6 +105,14 @@ __device__ __forceinline__ uint32_t low_bytes(uint32_t w0, uint32_t w1, uint32_t
     return __byte_perm(__byte_perm(w0, w1, 0x0040), __byte_perm(w2, w3, 0x0040), 0x5410);
 }
 
+// One 32-byte store (a whole L2 sector); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_v8(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                      uint32_t f, uint32_t g, uint32_t h) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(a), "r"(b), "r"(c), "r"(d),
+                 "r"(e), "r"(f), "r"(g), "r"(h)
+                 : "memory");
+}
+
 // Two codes (integers in [-8, 7], exact in e4m3) -> two e4m3 bytes: lo in
 // the low byte, hi in the high byte.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
@@ -450,6 +458,7 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
     constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer, half to even
     const float2 magic2 = make_float2(kMagic, kMagic);
     const bool divide = !p.unit_scales;
+    const bool v8_out = ((reinterpret_cast<uintptr_t>(p.qX) | reinterpret_cast<uintptr_t>(p.a8)) & 31u) == 0;
 
     for (int r = r0; r < p.rows; r += stride, ++it) {
         if (!keep) {
@@ -516,11 +525,19 @@ __global__ void __launch_bounds__(MAXT) act_kernel(ActArgs p) {
                 }
             }
         }
-        uint4* dq = reinterpret_cast<uint4*>(p.qX + (size_t)r * (K / 2) + (size_t)t * 32);
-        dq[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dq[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        {
-            uint4* d8 = reinterpret_cast<uint4*>(p.a8 + (size_t)r * K + (size_t)t * 64);
+        // whole 32-byte sectors per store where the bases allow it (K / 2 and the
+        // thread offsets are multiples of 32)
+        unsigned char* dqp = p.qX + (size_t)r * (K / 2) + (size_t)t * 32;
+        unsigned char* d8p = p.a8 + (size_t)r * K + (size_t)t * 64;
+        if (v8_out) {
+            st_v8(dqp, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+            st_v8(d8p, q8[0], q8[1], q8[2], q8[3], q8[4], q8[5], q8[6], q8[7]);
+            st_v8(d8p + 32, q8[8], q8[9], q8[10], q8[11], q8[12], q8[13], q8[14], q8[15]);
+        } else {
+            uint4* dq = reinterpret_cast<uint4*>(dqp);
+            dq[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dq[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            uint4* d8 = reinterpret_cast<uint4*>(d8p);
 #pragma unroll
             for (int i = 0; i < 4; ++i) d8[i] = make_uint4(q8[4 * i], q8[4 * i + 1], q8[4 * i + 2], q8[4 * i + 3]);
         }
