@@ -353,6 +353,40 @@ def test_activation_kernel_team_layouts(rrs, M, K):
     run_layer(rrs, X, W, wl.random_perm(K, M), 128, 2048, rows=np.unique(np.r_[0:4, M - 4:M, M // 2]))
 
 
+@pytest.mark.parametrize("misaligned", ["qX", "ws"])
+def test_activation_outputs_at_16_byte_offsets(rrs, misaligned):
+    """qX, or the workspace that holds the GEMM operand, 16- but not 32-byte aligned: the
+    activation kernel then writes with 16-byte stores instead of 32-byte ones; codes,
+    scales and the fp8 GEMM's Y are bit-identical to the aligned run."""
+    L = wl.LAYERS["llama3_8b_kv"]
+    M = 300
+    X = wl.make_activations(L, M=M).to(DEV)
+    perm = wl.random_perm(L.K, 5).to(DEV)
+    W = wl.make_weights(L).to(DEV)
+    qW, sw = rrs.prepare_weights(W, perm, L.had_block)
+    qW8 = rrs.expand_weights(qW)
+    flags = rrs.W_EXPANDED
+    n_ws = rrs.workspace_size(M, L.N, L.K, L.G, L.had_block, flags)
+
+    def run(qX_buf, ws_buf):
+        qX, s, st = rrs.smooth_quant(X, perm, L.G, L.had_block, flags=flags, qX=qX_buf, ws=ws_buf)
+        Y = rrs.w4a4_gemm(qX, s, st, qW8, sw, L.G, ws=ws_buf, flags=flags | rrs.WS_HOLDS_A8)
+        return qX.clone(), s.clone(), st.clone(), Y
+
+    ref = run(torch.empty((M, L.K // 2), dtype=torch.uint8, device=DEV),
+              torch.zeros(n_ws, dtype=torch.uint8, device=DEV))
+    qbuf = torch.empty(M * (L.K // 2) + 32, dtype=torch.uint8, device=DEV)
+    wbuf = torch.zeros(n_ws + 32, dtype=torch.uint8, device=DEV)
+    assert qbuf.data_ptr() % 32 == 0 and wbuf.data_ptr() % 32 == 0
+    qX_u = qbuf[16:16 + M * (L.K // 2)].view(M, L.K // 2) if misaligned == "qX" else qbuf[:M * (L.K // 2)].view(M, L.K // 2)
+    ws_u = wbuf[16:16 + n_ws] if misaligned == "ws" else wbuf[:n_ws]
+    got = run(qX_u, ws_u)
+    torch.cuda.synchronize()
+    for a, b, what in zip(got, ref, ("qX", "s", "scale_t", "Y")):
+        assert torch.equal(a.view(torch.uint8) if a.dtype == torch.uint8 else a.view(torch.int32),
+                           b.view(torch.uint8) if b.dtype == torch.uint8 else b.view(torch.int32)), what
+
+
 def test_zero_group_and_zero_token(rrs):
     L = wl.Layer("zeros", 40, 512, 256, 128, 512, seed=3)
     X, W = wl.make_activations(L), wl.make_weights(L)
