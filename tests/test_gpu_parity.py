@@ -421,18 +421,12 @@ def _sample_rows(M, st, k=48, seed=0):
 
 @pytest.mark.parametrize("name", ["llama3_8b_kv", "llama3_8b_qo", "llama3_8b_gateup", "llama3_8b_down"])
 def test_llama3_8b_layers(rrs, name):
-    """Every code and scale; Y on every row for q/o and k/v (the oracle's rows in
-    worker processes), on sampled rows (the largest-scale tokens among them) for the
-    wider gate/up and down layers."""
+    """Every code and scale, and Y on every row (the oracle's rows in worker
+    processes), at the full LLaMA-3-8B projection sizes."""
     L = wl.LAYERS[name]
     X, W = wl.make_activations(L), wl.make_weights(L)
     perm = torch.from_numpy(oracle.calibrate_perm(wl.make_activations(L, sample=1, M=512), L.had_block))
-    if L.N <= 4096 and L.K <= 4096:
-        run_layer(rrs, X, W, perm, L.G, L.had_block, rows=None, pool=True)
-        return
-    _, _, _, ost = oracle.smooth_quant(X, L.G, L.had_block, perm.numpy())
-    rows = _sample_rows(L.M, ost, k=24 if L.N > 8192 else 48)
-    run_layer(rrs, X, W, perm, L.G, L.had_block, rows=rows)
+    run_layer(rrs, X, W, perm, L.G, L.had_block, rows=None, pool=True)
 
 
 @pytest.mark.parametrize("name,N", [("llama3_70b_qo_decode_m1", 8192), ("llama3_70b_gateup_decode_m8", 4096),
